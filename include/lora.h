@@ -1,0 +1,176 @@
+/*
+ * lora.h - C ABI of the B200 (sm_100a) fused LoRA linear layer library.
+ *
+ * The layer (fastaf 0.1.0, "Minimal LoRA fine-tuning with hand-written
+ * Triton kernels", section "FWD kernel speedup"):
+ *
+ *     Y = X W^T + s (X A^T) B^T,        s = alpha / r
+ *
+ * its backward for a frozen W (same page, section "BWD kernel speedup",
+ * which names the dA, dB and dX kernels; the formulas follow from the
+ * forward by the chain rule), with T = X A^T recomputed:
+ *
+ *     dT = s dY B,   dB = s dY^T T,   dA = dT^T X,   dX = dY W + dT A
+ *
+ * and the adapter merge of the unsloth fork commit log
+ * (scripts/benchmarks/qwen3_flex_inference.py, the commit replacing
+ * copy + merge_adapter by one addmm(pristine, B, A, alpha=scaling)):
+ *
+ *     W_dst = W_src + s B A      (fp32 accumulate, one rounding to bf16)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are bf16 (passed as raw bit buffers), row-major, contiguous:
+ *   X[M, d_in], W[d_out, d_in], A[r, d_in], B[d_out, r], Y[M, d_out],
+ *   dY[M, d_out], dX[M, d_in], dA[r, d_in], dB[d_out, r].
+ * - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *   16-byte aligned.  Pointers to tensors with a zero-sized M dimension
+ *   (X, Y, dY, dX, and the workspace) may be NULL when M == 0.  The caller allocates and owns every buffer and the
+ *   stream; the library allocates no device memory of its own.
+ * - d_in and d_out are multiples of 8 (16-byte row pitch); r is a multiple
+ *   of 8 in [8, 128]; M >= 0 (M = 0 is a no-op).  Row counts need not be
+ *   multiples of any tile size.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *   asynchronous with respect to the host and ordered on `stream`.
+ * - s = alpha / r is computed in fp32 on the host.
+ * - Outputs must not overlap inputs, except W_dst == W_src in lora_merge.
+ * - Argument errors are returned before anything is launched and leave no
+ *   side effects.  A failed launch returns LORA_ERR_CUDA.  Kernels bound
+ *   every wait; a wait that runs out sets a device-side status word that
+ *   lora_get_device_status() reports (LORA_ERR_TIMEOUT).
+ * - Only sm_100 devices (B200) are supported; others get
+ *   LORA_ERR_UNSUPPORTED_DEVICE.
+ * - Calls on different streams may run concurrently; the library keeps no
+ *   per-call state besides the per-device status word.
+ */
+#ifndef LORA_B200_H
+#define LORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LORA_ABI_VERSION 1
+
+typedef enum {
+  LORA_OK = 0,
+  LORA_ERR_NULL = 1,               /* a required pointer is NULL */
+  LORA_ERR_SHAPE = 2,              /* negative size, or d_in/d_out not a multiple of 8 */
+  LORA_ERR_ALIGN = 3,              /* a pointer is not 16-byte aligned */
+  LORA_ERR_RANK = 4,               /* r not a multiple of 8 in [8, 128] */
+  LORA_ERR_WORKSPACE = 5,          /* workspace NULL or smaller than required */
+  LORA_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed */
+  LORA_ERR_TIMEOUT = 7,            /* a kernel gave up on a bounded wait */
+  LORA_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not sm_100 */
+  LORA_ERR_ALIAS = 9               /* an output overlaps an input */
+} lora_status_t;
+
+/* ABI version of the loaded library (LORA_ABI_VERSION it was built with). */
+int lora_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* lora_status_string(lora_status_t status);
+
+/*
+ * Forward: Y = X W^T + s (X A^T) B^T, rounded once to bf16.
+ *   X[M, d_in], W[d_out, d_in], A[r, d_in], B[d_out, r] in; Y[M, d_out] out.
+ * The [M, r] down-projection T = X A^T stays on chip: it is accumulated in
+ * tensor memory beside the base product, scaled by s and rounded to bf16
+ * (as an unfused bf16 X @ A.T would be), and fed to the up-projection,
+ * which accumulates onto the base product before the single store of Y.
+ */
+lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y,
+                       int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                       void* stream);
+
+/*
+ * Bytes of device scratch lora_bwd needs for this shape (0 when M == 0).
+ * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16) and the
+ * fp32 split-M partial sums of dA and dB.
+ */
+size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r);
+
+/*
+ * Backward for frozen W:
+ *   dX[M, d_in]  = dY W + dT A       (bf16)
+ *   dA[r, d_in]  = dT^T X            (bf16, reduced over M in fp32)
+ *   dB[d_out, r] = s dY^T T          (bf16, reduced over M in fp32)
+ * with T = X A^T recomputed and dT = s dY B (rounded to bf16 on chip).
+ * `workspace` is caller-owned device memory of at least
+ * lora_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on
+ * entry do not matter and are clobbered.  Results are bitwise repeatable:
+ * the M reduction of dA and dB uses fixed-order partial sums, no atomics.
+ * With M == 0, dA and dB are set to zero and nothing else happens.
+ */
+lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B,
+                       const void* dY, void* dX, void* dA, void* dB,
+                       int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Merge: W_dst[d_out, d_in] = bf16_rne(W_src + s * (B A)), the rank-r
+ * product accumulated in fp32 and rounded once.  W_src is the pristine base
+ * (restore + merge in one pass) or W_dst itself (in place).
+ * A[r, d_in], B[d_out, r].
+ */
+lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst,
+                         int64_t d_out, int64_t d_in, int32_t r, float alpha, void* stream);
+
+/* One matrix of a batched merge (all pointers device pointers). */
+typedef struct {
+  const void* W_src;
+  const void* A;
+  const void* B;
+  void* W_dst;
+  int64_t d_out;
+  int64_t d_in;
+} lora_merge_desc_t;
+
+/*
+ * Batched merge of n matrices sharing r and alpha (e.g. every LoRA target of
+ * a model), one persistent launch.  `descs` is a HOST array of n entries,
+ * read during the call.  Each entry follows lora_merge's rules.
+ */
+lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int32_t r,
+                                 float alpha, void* stream);
+
+/*
+ * Restore: W_dst <- W_src, a bit copy of n_elems bf16 values (the pristine
+ * copy is only read).
+ */
+lora_status_t lora_restore(const void* W_src, void* W_dst, int64_t n_elems, void* stream);
+
+/*
+ * Synchronizes the current device, returns LORA_ERR_TIMEOUT if any kernel
+ * of this library gave up on a bounded wait since the last call (and clears
+ * the flag), LORA_ERR_CUDA on a CUDA error, else LORA_OK.
+ */
+lora_status_t lora_get_device_status(void);
+
+/*
+ * Host-only validation (no GPU needed): checks pointers and sizes exactly as
+ * the entry point for `op` would (op 0 = lora_fwd with ptrs {X,W,A,B,Y};
+ * 1 = lora_bwd with {X,W,A,B,dY,dX,dA,dB,workspace}; 2 = lora_merge with
+ * {W_src,A,B,W_dst}; M is ignored for op 2).  `workspace_bytes` is only
+ * read for op 1.
+ */
+lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptrs,
+                              int64_t M, int64_t d_in, int64_t d_out, int32_t r,
+                              size_t workspace_bytes);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one block that waits on
+ * a barrier nothing will arrive on, with the given limit in nanoseconds
+ * (clamped to [1e3, 1e9]).  Returns what lora_get_device_status() then
+ * reports: LORA_ERR_TIMEOUT when the wait gave up as designed.
+ */
+lora_status_t lora_selftest_wait_timeout(int64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_B200_H */

@@ -1,0 +1,222 @@
+"""Python binding of the B200 fused LoRA linear layer library.
+
+Argument marshalling only: each function takes torch CUDA tensors (bf16,
+contiguous), passes their device pointers, sizes and the current CUDA stream
+to the C ABI of ``include/lora.h`` (``_lib/liblora_b200.so``) and raises
+``LoraError`` on a non-OK status.  Every step of the layer runs in the
+library's kernels; there is no fallback of any kind.  If the shared library
+is missing, the first call raises ``LoraLibraryMissing``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "liblora_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lora.h")
+
+STATUS = {
+    0: "LORA_OK", 1: "LORA_ERR_NULL", 2: "LORA_ERR_SHAPE", 3: "LORA_ERR_ALIGN",
+    4: "LORA_ERR_RANK", 5: "LORA_ERR_WORKSPACE", 6: "LORA_ERR_CUDA",
+    7: "LORA_ERR_TIMEOUT", 8: "LORA_ERR_UNSUPPORTED_DEVICE", 9: "LORA_ERR_ALIAS",
+}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+
+class LoraError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = int(code)
+        super().__init__(f"{what}: {STATUS.get(self.code, self.code)} ({lora_status_string(self.code)})")
+
+
+class LoraLibraryMissing(ImportError):
+    pass
+
+
+class _MergeDesc(ctypes.Structure):
+    _fields_ = [("W_src", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("W_dst", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64)]
+
+
+_lib_handle = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load (once) and return the shared library; raise if it is missing."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    with _lock:
+        if _lib_handle is not None:
+            return _lib_handle
+        if not os.path.exists(LIB_PATH):
+            raise LoraLibraryMissing(
+                f"{LIB_PATH} not found: build it with lora_linear_layer_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, i32, f32, vp, sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+        L.lora_abi_version.restype = ctypes.c_int
+        L.lora_abi_version.argtypes = []
+        L.lora_status_string.restype = ctypes.c_char_p
+        L.lora_status_string.argtypes = [ctypes.c_int]
+        L.lora_fwd.restype = ctypes.c_int
+        L.lora_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
+        L.lora_bwd_workspace_size.restype = sz
+        L.lora_bwd_workspace_size.argtypes = [i64, i64, i64, i32]
+        L.lora_bwd.restype = ctypes.c_int
+        L.lora_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, vp]
+        L.lora_merge.restype = ctypes.c_int
+        L.lora_merge.argtypes = [vp, vp, vp, vp, i64, i64, i32, f32, vp]
+        L.lora_merge_batched.restype = ctypes.c_int
+        L.lora_merge_batched.argtypes = [ctypes.POINTER(_MergeDesc), i32, i32, f32, vp]
+        L.lora_restore.restype = ctypes.c_int
+        L.lora_restore.argtypes = [vp, vp, i64, vp]
+        L.lora_get_device_status.restype = ctypes.c_int
+        L.lora_get_device_status.argtypes = []
+        L.lora_check_args.restype = ctypes.c_int
+        L.lora_check_args.argtypes = [i32, ctypes.POINTER(vp), i32, i64, i64, i64, i32, sz]
+        L.lora_selftest_wait_timeout.restype = ctypes.c_int
+        L.lora_selftest_wait_timeout.argtypes = [i64]
+        _lib_handle = L
+        return L
+
+
+# ------------------------------------------------------------ helpers ----
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check_tensor(t, name: str, shape: Optional[Tuple[int, ...]] = None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bf16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _raise(code: int, what: str):
+    if code != 0:
+        raise LoraError(code, what)
+
+
+# --------------------------------------------------------------- ABI ----
+
+def lora_abi_version() -> int:
+    return int(lib().lora_abi_version())
+
+
+def lora_status_string(code: int) -> str:
+    return lib().lora_status_string(int(code)).decode()
+
+
+def lora_fwd(X, W, A, B, Y, alpha: float, stream=None) -> None:
+    """Y = X W^T + (alpha/r) (X A^T) B^T (see include/lora.h)."""
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
+        _check_tensor(t, n, s)
+    code = lib().lora_fwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r,
+                          float(alpha), _stream(stream))
+    _raise(code, "lora_fwd")
+
+
+def lora_bwd_workspace_size(M: int, d_in: int, d_out: int, r: int) -> int:
+    return int(lib().lora_bwd_workspace_size(int(M), int(d_in), int(d_out), int(r)))
+
+
+def lora_bwd(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, stream=None) -> None:
+    """dX = dY W + dT A, dA = dT^T X, dB = s dY^T T (see include/lora.h).
+
+    ``workspace`` is a CUDA tensor (any dtype) of at least
+    ``lora_bwd_workspace_size(M, d_in, d_out, r)`` bytes."""
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r)), (dY, "dY", (M, d_out)), (dX, "dX", (M, d_in)),
+                    (dA, "dA", (r, d_in)), (dB, "dB", (d_out, r))):
+        _check_tensor(t, n, s)
+    ws_bytes = int(workspace.numel() * workspace.element_size())
+    code = lib().lora_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
+                          M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(code, "lora_bwd")
+
+
+def lora_merge(W_src, A, B, W_dst, alpha: float, stream=None) -> None:
+    """W_dst = bf16(W_src + (alpha/r) B A); W_dst may be W_src (in place)."""
+    d_out, d_in = W_src.shape
+    r = A.shape[0]
+    for t, n, s in ((W_src, "W_src", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
+                    (W_dst, "W_dst", (d_out, d_in))):
+        _check_tensor(t, n, s)
+    code = lib().lora_merge(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in, r, float(alpha),
+                            _stream(stream))
+    _raise(code, "lora_merge")
+
+
+def lora_merge_batched(items: Sequence[Tuple], r: int, alpha: float, stream=None) -> None:
+    """Merge every (W_src, A, B, W_dst) of ``items`` (shared r, alpha)."""
+    n = len(items)
+    arr = (_MergeDesc * max(n, 1))()
+    for i, (W_src, A, B, W_dst) in enumerate(items):
+        d_out, d_in = W_src.shape
+        for t, nm, s in ((W_src, "W_src", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
+                         (W_dst, "W_dst", (d_out, d_in))):
+            _check_tensor(t, nm, s)
+        arr[i] = _MergeDesc(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in)
+    code = lib().lora_merge_batched(arr, n, int(r), float(alpha), _stream(stream))
+    _raise(code, "lora_merge_batched")
+
+
+def lora_restore(W_src, W_dst, stream=None) -> None:
+    """W_dst <- W_src (bit copy)."""
+    _check_tensor(W_src, "W_src")
+    _check_tensor(W_dst, "W_dst", tuple(W_src.shape))
+    code = lib().lora_restore(_ptr(W_src), _ptr(W_dst), W_src.numel(), _stream(stream))
+    _raise(code, "lora_restore")
+
+
+def lora_get_device_status() -> int:
+    """Synchronize the device; return the status code (0 = OK)."""
+    return int(lib().lora_get_device_status())
+
+
+def lora_check_args(op: int, ptrs: Sequence[int], M: int, d_in: int, d_out: int, r: int,
+                    workspace_bytes: int = 0) -> int:
+    """Host-only validation (no GPU): returns the status code."""
+    n = len(ptrs)
+    arr = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(p) if p else None for p in ptrs])
+    return int(lib().lora_check_args(int(op), arr, n, int(M), int(d_in), int(d_out), int(r),
+                                     int(workspace_bytes)))
+
+
+def lora_selftest_wait_timeout(limit_ns: int) -> int:
+    return int(lib().lora_selftest_wait_timeout(int(limit_ns)))
+
+
+def header_functions() -> list:
+    """Names of the functions include/lora.h declares (for export checks)."""
+    import re
+    with open(HEADER_PATH) as f:
+        txt = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\**\s+\**(lora_[a-z0-9_]+)\s*\(",
+                                 txt, flags=re.M)))

@@ -1,0 +1,652 @@
+// lora_api.cu - the extern "C" entry points declared in include/lora.h.
+//
+// Host side of the library: argument validation, TMA tensor-map encoding,
+// tile / pipeline configuration and kernel launches on the caller's stream.
+// All arithmetic of the layer runs in the kernels of fused.cuh, skinny.cuh
+// and merge.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lora.h"
+#include "common.cuh"
+#include "fused.cuh"
+#include "merge.cuh"
+#include "skinny.cuh"
+
+namespace lora {
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(smem_addr(&bar), 0u, &abort_flag, limit_ns, SITE_SELFTEST);
+  __syncthreads();
+}
+
+}  // namespace lora
+
+namespace {
+
+using namespace lora;
+
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitimate wait
+constexpr uint32_t kSmemMax = 232448;             // 227 KB opt-in dynamic shared memory
+constexpr int kSplitSMs = 148;                    // B200 SM count used to size split-M work
+
+// ------------------------------------------------------------ validation ----
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range range_of(const void* p, uint64_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return Range{a, a + bytes};
+}
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+lora_status_t check_sizes(int64_t M, int64_t d_in, int64_t d_out, int32_t r) {
+  if (M < 0 || d_in <= 0 || d_out <= 0) return LORA_ERR_SHAPE;
+  if ((d_in % 8) != 0 || (d_out % 8) != 0) return LORA_ERR_SHAPE;
+  if (M > (int64_t(1) << 30) || d_in > (int64_t(1) << 30) || d_out > (int64_t(1) << 30)) return LORA_ERR_SHAPE;
+  if (r < 8 || r > 128 || (r % 8) != 0) return LORA_ERR_RANK;
+  return LORA_OK;
+}
+
+int r_pad_of(int r) { return (r + 15) / 16 * 16; }
+int rcw_of(int r_pad) { return r_pad <= 16 ? 16 : r_pad <= 32 ? 32 : 64; }
+
+// ---------------------------------------------------------- device state ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+EncodeTiledFn g_encode = nullptr;
+
+lora_status_t device_info(DeviceInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LORA_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    d.probed = true;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return LORA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  out = d;
+  return d.supported ? LORA_OK : LORA_ERR_UNSUPPORTED_DEVICE;
+}
+
+CUtensorMapSwizzle swz_enum(uint32_t span_bytes) {
+  return span_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+         : span_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                            : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
+// row pitch `ld` elements, box {box_inner, box_outer}.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
+              uint32_t box_outer, uint32_t swz_span_bytes) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult rc = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz_enum(swz_span_bytes),
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (rc != CUDA_SUCCESS) {
+    std::fprintf(stderr, "lora_b200: cuTensorMapEncodeTiled failed (%d) dims=%llu,%llu box=%u,%u\n", int(rc),
+                 (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+    return false;
+  }
+  return true;
+}
+
+lora_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "lora_b200: launch failed: %s\n", cudaGetErrorString(e));
+    return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
+}
+
+// ------------------------------------------------------------ fused GEMM ----
+
+struct FusedCfg {
+  int BN, RCW, r_pad, n_rchunks, stages, grid;
+  uint32_t smem;
+  FusedArgs args;
+};
+
+bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, FusedCfg& c) {
+  c.r_pad = r_pad_of(r);
+  c.RCW = rcw_of(c.r_pad);
+  c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
+  const int num_m = int((M + kBM - 1) / kBM);
+  const int cands[2] = {256, 128};
+  c.BN = 0;
+  for (int BN : cands) {
+    const FusedLayout L0(BN, mn, c.RCW, c.r_pad, c.n_rchunks, 0);
+    const uint32_t fixed = L0.total + 1024;
+    if (fixed >= kSmemMax) continue;
+    int S = int((kSmemMax - fixed) / L0.stage_bytes);
+    S = std::min(S, 8);
+    const int num_n = int((N + BN - 1) / BN);
+    const bool enough_tiles = (int64_t)num_m * num_n >= sm_count;
+    if (BN == 256 && (S < 3 || !enough_tiles)) continue;
+    if (S < 2) continue;
+    c.BN = BN;
+    c.stages = S;
+    break;
+  }
+  if (c.BN == 0) return false;
+  const int num_n = int((N + c.BN - 1) / c.BN);
+  const FusedLayout L(c.BN, mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
+  c.smem = L.total + 1024;
+  FusedArgs& a = c.args;
+  a.M = int32_t(M);
+  a.N = int32_t(N);
+  a.K = int32_t(K);
+  a.r_pad = c.r_pad;
+  a.n_rchunks = c.n_rchunks;
+  a.stages = c.stages;
+  a.num_m = num_m;
+  a.num_n = num_n;
+  // Column bands keep the operands the whole GPU touches at once well
+  // inside the 126 MB L2 when the full problem is larger than that.
+  const double footprint = double(M + N) * double(K) * 2.0;
+  if (footprint > 96.0e6) {
+    const double per_ntile = double(c.BN) * double(K) * 2.0;
+    a.band_w = std::max(1, std::min(num_n, int(40.0e6 / per_ntile)));
+  } else {
+    a.band_w = num_n;
+  }
+  a.n_bands = (num_n + a.band_w - 1) / a.band_w;
+  a.wait_limit_ns = kWaitLimitNs;
+  c.grid = int(std::min<int64_t>(sm_count, (int64_t)num_m * num_n));
+  return true;
+}
+
+template <int BN, bool MN, int RCW>
+lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, cudaStream_t st) {
+  auto kern = fused_lora_kernel<BN, MN, RCW>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
+    return LORA_ERR_CUDA;
+  kern<<<c.grid, kFusedThreads, c.smem, st>>>(maps[0], maps[1], maps[2], maps[3], c.args);
+  return launch_status();
+}
+
+template <bool MN>
+lora_status_t launch_fused(const CUtensorMap* maps, const FusedCfg& c, cudaStream_t st) {
+  if (c.BN == 256) {
+    if (c.RCW == 16) return launch_fused_t<256, MN, 16>(maps, c, st);
+    if (c.RCW == 32) return launch_fused_t<256, MN, 32>(maps, c, st);
+    return launch_fused_t<256, MN, 64>(maps, c, st);
+  }
+  if (c.RCW == 16) return launch_fused_t<128, MN, 16>(maps, c, st);
+  if (c.RCW == 32) return launch_fused_t<128, MN, 32>(maps, c, st);
+  return launch_fused_t<128, MN, 64>(maps, c, st);
+}
+
+// ----------------------------------------------------------- skinny GEMM ----
+
+struct SkinnyCfg {
+  int RCW, r_pad, n_rchunks, stages, splits;
+  uint32_t smem;
+  SkinnyArgs args;
+};
+
+void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, bool split, SkinnyCfg& c) {
+  c.r_pad = r_pad_of(r);
+  c.RCW = rcw_of(c.r_pad);
+  c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
+  c.stages = 4;
+  const int row_tiles = int((rows + 127) / 128);
+  const int nk = int((K + 63) / 64);
+  int splits = 1;
+  if (split) {
+    const int target = 2 * kSplitSMs;
+    splits = std::max(1, std::min((target + row_tiles - 1) / row_tiles, std::max(1, nk / 4)));
+  }
+  const int kb_per = std::max(1, (nk + splits - 1) / splits);
+  splits = std::max(1, (nk + kb_per - 1) / kb_per);
+  c.splits = splits;
+  const SkinnyLayout L(r_mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
+  c.smem = L.total + 1024;
+  SkinnyArgs& a = c.args;
+  a.rows = int32_t(rows);
+  a.K = int32_t(K);
+  a.r_pad = c.r_pad;
+  a.n_rchunks = c.n_rchunks;
+  a.stages = c.stages;
+  a.kb_per_split = kb_per;
+  a.scale = 1.0f;
+  a.out_bf16 = nullptr;
+  a.out_f32 = nullptr;
+  a.wait_limit_ns = kWaitLimitNs;
+}
+
+template <bool P_MN, bool R_MN, bool PARTIALS, int RCW>
+lora_status_t launch_skinny_t(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
+  auto kern = skinny_kernel<P_MN, R_MN, RCW, PARTIALS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
+    return LORA_ERR_CUDA;
+  dim3 grid(unsigned((c.args.rows + 127) / 128), unsigned(c.splits));
+  kern<<<grid, 192, c.smem, st>>>(p, rm, c.args);
+  return launch_status();
+}
+
+template <bool P_MN, bool R_MN, bool PARTIALS>
+lora_status_t launch_skinny(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
+  if (c.RCW == 16) return launch_skinny_t<P_MN, R_MN, PARTIALS, 16>(p, rm, c, st);
+  if (c.RCW == 32) return launch_skinny_t<P_MN, R_MN, PARTIALS, 32>(p, rm, c, st);
+  return launch_skinny_t<P_MN, R_MN, PARTIALS, 64>(p, rm, c, st);
+}
+
+// --------------------------------------------------------- bwd workspace ----
+
+struct BwdPlan {
+  SkinnyCfg t_cfg, db_cfg, da_cfg;
+  size_t off_t, off_dt, off_pb, off_pa, total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
+  pick_skinny(M, d_in, r, false, false, p.t_cfg);
+  pick_skinny(d_out, M, r, true, true, p.db_cfg);
+  pick_skinny(d_in, M, r, true, true, p.da_cfg);
+  const int r_pad = r_pad_of(r);
+  const size_t tb = align256(size_t(M) * r_pad * 2);
+  p.off_t = 0;
+  p.off_dt = tb;
+  p.off_pb = 2 * tb;
+  p.off_pa = p.off_pb + align256(size_t(p.db_cfg.splits) * size_t(d_out) * r_pad * 4);
+  p.total = p.off_pa + align256(size_t(p.da_cfg.splits) * size_t(d_in) * r_pad * 4);
+}
+
+// -------------------------------------------------------- merge batching ----
+
+struct MergeItem {
+  const void* W_src;
+  const void* A;
+  const void* B;
+  void* W_dst;
+  int64_t d_out, d_in;
+};
+
+lora_status_t check_merge_item(const MergeItem& it, int32_t r) {
+  if (!it.W_src || !it.A || !it.B || !it.W_dst) return LORA_ERR_NULL;
+  lora_status_t s = check_sizes(0, it.d_in, it.d_out, r);
+  if (s != LORA_OK) return s;
+  if (!aligned16(it.W_src) || !aligned16(it.A) || !aligned16(it.B) || !aligned16(it.W_dst)) return LORA_ERR_ALIGN;
+  const Range dst = range_of(it.W_dst, uint64_t(it.d_out) * it.d_in * 2);
+  if (overlaps(dst, range_of(it.A, uint64_t(r) * it.d_in * 2)) ||
+      overlaps(dst, range_of(it.B, uint64_t(it.d_out) * r * 2)))
+    return LORA_ERR_ALIAS;
+  if (it.W_dst != it.W_src && overlaps(dst, range_of(it.W_src, uint64_t(it.d_out) * it.d_in * 2)))
+    return LORA_ERR_ALIAS;
+  return LORA_OK;
+}
+
+template <int RCW>
+lora_status_t launch_merge_t(const MergeTable& tab, int total_tiles, uint32_t smem, cudaStream_t st) {
+  auto kern = merge_kernel<RCW>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    return LORA_ERR_CUDA;
+  kern<<<total_tiles, 192, smem, st>>>(tab);
+  return launch_status();
+}
+
+lora_status_t run_merge(const MergeItem* items, int n, int32_t r, float alpha, cudaStream_t st) {
+  if (n <= 0) return LORA_OK;
+  const int r_pad = r_pad_of(r);
+  const int rcw = rcw_of(r_pad);
+  const int n_rchunks = (r_pad + rcw - 1) / rcw;
+  const MergeLayout L(rcw, r_pad, n_rchunks);
+  const uint32_t smem = L.total + 1024;
+  static thread_local MergeTable tab;  // ~28 KB, kept off the stack
+  int i = 0;
+  while (i < n) {
+    std::memset(&tab, 0, sizeof(tab));
+    tab.r_pad = r_pad;
+    tab.n_rchunks = n_rchunks;
+    tab.scale = alpha / float(r);
+    tab.wait_limit_ns = kWaitLimitNs;
+    int tiles = 0, nj = 0;
+    for (; i < n && nj < kMergeMaxJobs; ++i) {
+      const MergeItem& it = items[i];
+      MergeJob& j = tab.job[nj];
+      if (!make_map(&j.w_src, it.W_src, it.d_in, it.d_out, it.d_in, 64, 128, 128) ||
+          !make_map(&j.w_dst, it.W_dst, it.d_in, it.d_out, it.d_in, 64, 32, 128) ||
+          !make_map(&j.a, it.A, it.d_in, r, it.d_in, 64, r_pad, 128) ||
+          !make_map(&j.b, it.B, r, it.d_out, r, rcw, 128, rcw * 2))
+        return LORA_ERR_CUDA;
+      j.tiles_n = int32_t((it.d_in + kMergeBN - 1) / kMergeBN);
+      j.tile_begin = tiles;
+      tiles += j.tiles_n * int32_t((it.d_out + 127) / 128);
+      ++nj;
+    }
+    tab.n_jobs = nj;
+    lora_status_t s = rcw == 16 ? launch_merge_t<16>(tab, tiles, smem, st)
+                      : rcw == 32 ? launch_merge_t<32>(tab, tiles, smem, st)
+                                  : launch_merge_t<64>(tab, tiles, smem, st);
+    if (s != LORA_OK) return s;
+  }
+  return LORA_OK;
+}
+
+lora_status_t zero_bytes(void* p, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return LORA_OK;
+  if ((bytes % 16) != 0 || !aligned16(p)) return LORA_ERR_ALIGN;
+  const size_t n16 = bytes / 16;
+  const int blocks = int(std::min<size_t>((n16 + 255) / 256, 4096));
+  zero16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<uint4*>(p), n16);
+  return launch_status();
+}
+
+}  // namespace
+
+// ================================================================ C ABI ====
+
+extern "C" {
+
+int lora_abi_version(void) { return LORA_ABI_VERSION; }
+
+const char* lora_status_string(lora_status_t s) {
+  switch (s) {
+    case LORA_OK: return "LORA_OK";
+    case LORA_ERR_NULL: return "LORA_ERR_NULL: a required pointer is NULL";
+    case LORA_ERR_SHAPE: return "LORA_ERR_SHAPE: bad size (d_in, d_out must be positive multiples of 8)";
+    case LORA_ERR_ALIGN: return "LORA_ERR_ALIGN: pointer not 16-byte aligned";
+    case LORA_ERR_RANK: return "LORA_ERR_RANK: r must be a multiple of 8 in [8, 128]";
+    case LORA_ERR_WORKSPACE: return "LORA_ERR_WORKSPACE: workspace missing or too small";
+    case LORA_ERR_CUDA: return "LORA_ERR_CUDA: a CUDA call failed";
+    case LORA_ERR_TIMEOUT: return "LORA_ERR_TIMEOUT: a kernel gave up on a bounded wait";
+    case LORA_ERR_UNSUPPORTED_DEVICE: return "LORA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
+    case LORA_ERR_ALIAS: return "LORA_ERR_ALIAS: an output overlaps an input";
+  }
+  return "LORA_ERR_UNKNOWN";
+}
+
+lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in,
+                              int64_t d_out, int32_t r, size_t workspace_bytes) {
+  if (op == 0) {
+    // X and Y may be NULL only when M == 0 (nothing is read or written).
+    if (ptrs == nullptr || n_ptrs != 5) return LORA_ERR_NULL;
+    for (int i = 0; i < 5; ++i) {
+      const bool needed = (i >= 1 && i <= 3) || M != 0;
+      if (needed && ptrs[i] == nullptr) return LORA_ERR_NULL;
+    }
+    lora_status_t s = check_sizes(M, d_in, d_out, r);
+    if (s != LORA_OK) return s;
+    for (int i = 0; i < 5; ++i)
+      if (!aligned16(ptrs[i])) return LORA_ERR_ALIGN;
+    const Range y = range_of(ptrs[4], uint64_t(M) * d_out * 2);
+    if (overlaps(y, range_of(ptrs[0], uint64_t(M) * d_in * 2)) ||
+        overlaps(y, range_of(ptrs[1], uint64_t(d_out) * d_in * 2)) ||
+        overlaps(y, range_of(ptrs[2], uint64_t(r) * d_in * 2)) ||
+        overlaps(y, range_of(ptrs[3], uint64_t(d_out) * r * 2)))
+      return LORA_ERR_ALIAS;
+    return LORA_OK;
+  }
+  if (op == 1) {
+    // X, dY, dX (and the workspace) may be NULL only when M == 0; dA and dB
+    // are always written (zeros when M == 0).
+    if (ptrs == nullptr || n_ptrs != 9) return LORA_ERR_NULL;
+    for (int i = 0; i < 8; ++i) {
+      const bool needed = (i >= 1 && i <= 3) || i == 6 || i == 7 || M != 0;
+      if (needed && ptrs[i] == nullptr) return LORA_ERR_NULL;
+    }
+    lora_status_t s = check_sizes(M, d_in, d_out, r);
+    if (s != LORA_OK) return s;
+    for (int i = 0; i < 8; ++i)
+      if (!aligned16(ptrs[i])) return LORA_ERR_ALIGN;
+    const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
+    if (need > 0) {
+      if (ptrs[8] == nullptr || workspace_bytes < need) return LORA_ERR_WORKSPACE;
+      if ((reinterpret_cast<uintptr_t>(ptrs[8]) & 255u) != 0) return LORA_ERR_ALIGN;
+    }
+    const Range in[5] = {range_of(ptrs[0], uint64_t(M) * d_in * 2), range_of(ptrs[1], uint64_t(d_out) * d_in * 2),
+                         range_of(ptrs[2], uint64_t(r) * d_in * 2), range_of(ptrs[3], uint64_t(d_out) * r * 2),
+                         range_of(ptrs[4], uint64_t(M) * d_out * 2)};
+    const Range out[4] = {range_of(ptrs[5], uint64_t(M) * d_in * 2), range_of(ptrs[6], uint64_t(r) * d_in * 2),
+                          range_of(ptrs[7], uint64_t(d_out) * r * 2), range_of(ptrs[8], need)};
+    for (int o = 0; o < 4; ++o) {
+      for (int i = 0; i < 5; ++i)
+        if (overlaps(out[o], in[i])) return LORA_ERR_ALIAS;
+      for (int o2 = o + 1; o2 < 4; ++o2)
+        if (overlaps(out[o], out[o2])) return LORA_ERR_ALIAS;
+    }
+    return LORA_OK;
+  }
+  if (op == 2) {
+    if (ptrs == nullptr || n_ptrs != 4) return LORA_ERR_NULL;
+    MergeItem it{ptrs[0], ptrs[1], ptrs[2], const_cast<void*>(ptrs[3]), d_out, d_in};
+    return check_merge_item(it, r);
+  }
+  return LORA_ERR_SHAPE;
+}
+
+lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                       int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
+  const void* ptrs[5] = {X, W, A, B, Y};
+  lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
+  if (s != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  if (M == 0) return LORA_OK;
+  FusedCfg c;
+  if (!pick_fused(M, d_out, d_in, r, false, dev.sm_count, c)) return LORA_ERR_RANK;
+  c.args.scale = alpha / float(r);
+  c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
+  c.args.t_out = nullptr;
+  CUtensorMap maps[4];
+  if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
+      !make_map(&maps[1], W, d_in, d_out, d_in, 64, c.BN, 128) ||
+      !make_map(&maps[2], A, d_in, r, d_in, 64, c.r_pad, 128) ||
+      !make_map(&maps[3], B, r, d_out, r, c.RCW, c.BN, c.RCW * 2))
+    return LORA_ERR_CUDA;
+  return launch_fused<false>(maps, c, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r) {
+  if (check_sizes(M, d_in, d_out, r) != LORA_OK || M == 0) return 0;
+  BwdPlan p;
+  plan_bwd(M, d_in, d_out, r, p);
+  return p.total;
+}
+
+lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                       void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
+  lora_status_t s = lora_check_args(1, ptrs, 9, M, d_in, d_out, r, workspace_bytes);
+  if (s != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if ((s = zero_bytes(dA, size_t(r) * d_in * 2, st)) != LORA_OK) return s;
+    return zero_bytes(dB, size_t(d_out) * r * 2, st);
+  }
+  BwdPlan p;
+  plan_bwd(M, d_in, d_out, r, p);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_t);
+  __nv_bfloat16* dTws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_dt);
+  float* partB = reinterpret_cast<float*>(ws + p.off_pb);
+  float* partA = reinterpret_cast<float*>(ws + p.off_pa);
+  const float scale = alpha / float(r);
+  const int r_pad = r_pad_of(r);
+  const int rcw = rcw_of(r_pad);
+
+  // 1. T = X A^T (recomputed), bf16 [M, r_pad]
+  {
+    CUtensorMap mp, mr;
+    if (!make_map(&mp, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr, A, d_in, r, d_in, 64, r_pad, 128))
+      return LORA_ERR_CUDA;
+    SkinnyCfg c = p.t_cfg;
+    c.args.out_bf16 = Tws;
+    c.args.scale = 1.0f;
+    if ((s = launch_skinny<false, false, false>(mp, mr, c, st)) != LORA_OK) return s;
+  }
+  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad])
+  {
+    FusedCfg c;
+    if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
+    c.args.scale = scale;
+    c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
+    c.args.t_out = dTws;
+    CUtensorMap maps[4];
+    if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
+        !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
+        !make_map(&maps[2], B, r, d_out, r, rcw, 64, rcw * 2) ||
+        !make_map(&maps[3], A, d_in, r, d_in, 64, r_pad, 128))
+      return LORA_ERR_CUDA;
+    if ((s = launch_fused<true>(maps, c, st)) != LORA_OK) return s;
+  }
+  // 3. dB partials: sum_m dY[m, i] T[m, j]
+  {
+    CUtensorMap mp, mr;
+    if (!make_map(&mp, dY, d_out, M, d_out, 64, 64, 128) || !make_map(&mr, Tws, r_pad, M, r_pad, rcw, 64, rcw * 2))
+      return LORA_ERR_CUDA;
+    SkinnyCfg c = p.db_cfg;
+    c.args.out_f32 = partB;
+    if ((s = launch_skinny<true, true, true>(mp, mr, c, st)) != LORA_OK) return s;
+  }
+  // 4. dA^T partials: sum_m X[m, i] dT[m, j]
+  {
+    CUtensorMap mp, mr;
+    if (!make_map(&mp, X, d_in, M, d_in, 64, 64, 128) || !make_map(&mr, dTws, r_pad, M, r_pad, rcw, 64, rcw * 2))
+      return LORA_ERR_CUDA;
+    SkinnyCfg c = p.da_cfg;
+    c.args.out_f32 = partA;
+    if ((s = launch_skinny<true, true, true>(mp, mr, c, st)) != LORA_OK) return s;
+  }
+  // 5. fixed-order reductions: dB = s * sum, dA = (sum)^T
+  reduce_partials_kernel<<<unsigned((d_out + 31) / 32), 256, 0, st>>>(
+      partB, p.db_cfg.splits, int(d_out), r_pad, r, scale, reinterpret_cast<__nv_bfloat16*>(dB), 0);
+  if ((s = launch_status()) != LORA_OK) return s;
+  reduce_partials_kernel<<<unsigned((d_in + 31) / 32), 256, 0, st>>>(
+      partA, p.da_cfg.splits, int(d_in), r_pad, r, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), 1);
+  return launch_status();
+}
+
+lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
+                         int64_t d_in, int32_t r, float alpha, void* stream) {
+  MergeItem it{W_src, A, B, W_dst, d_out, d_in};
+  lora_status_t s = check_merge_item(it, r);
+  if (s != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  return run_merge(&it, 1, r, alpha, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
+  if (n < 0) return LORA_ERR_SHAPE;
+  if (n == 0) return LORA_OK;
+  if (descs == nullptr) return LORA_ERR_NULL;
+  std::vector<MergeItem> items(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    items[i] = MergeItem{descs[i].W_src, descs[i].A, descs[i].B, descs[i].W_dst, descs[i].d_out, descs[i].d_in};
+    lora_status_t s = check_merge_item(items[i], r);
+    if (s != LORA_OK) return s;
+  }
+  DeviceInfo dev;
+  lora_status_t s = device_info(dev);
+  if (s != LORA_OK) return s;
+  return run_merge(items.data(), n, r, alpha, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lora_status_t lora_restore(const void* W_src, void* W_dst, int64_t n_elems, void* stream) {
+  if (n_elems < 0) return LORA_ERR_SHAPE;
+  if (n_elems == 0) return LORA_OK;
+  if (!W_src || !W_dst) return LORA_ERR_NULL;
+  if (!aligned16(W_src) || !aligned16(W_dst)) return LORA_ERR_ALIGN;
+  if (W_src != W_dst && overlaps(range_of(W_src, uint64_t(n_elems) * 2), range_of(W_dst, uint64_t(n_elems) * 2)))
+    return LORA_ERR_ALIAS;
+  DeviceInfo dev;
+  lora_status_t s = device_info(dev);
+  if (s != LORA_OK) return s;
+  if (W_src == W_dst) return LORA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t n16 = size_t(n_elems) * 2 / 16;
+  if (n16 > 0) {
+    const int blocks = int(std::min<size_t>((n16 + 255) / 256, size_t(dev.sm_count) * 8));
+    copy16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(W_src), reinterpret_cast<uint4*>(W_dst), n16);
+    if ((s = launch_status()) != LORA_OK) return s;
+  }
+  const size_t done = n16 * 8;
+  const size_t rest = size_t(n_elems) - done;
+  if (rest > 0) {
+    copy2_kernel<<<1, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(W_src) + done,
+                                    reinterpret_cast<uint16_t*>(W_dst) + done, rest);
+    if ((s = launch_status()) != LORA_OK) return s;
+  }
+  return LORA_OK;
+}
+
+lora_status_t lora_get_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return LORA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lora::g_status, sizeof(v)) != cudaSuccess) return LORA_ERR_CUDA;
+  if (v != 0u) {
+    unsigned int info[4] = {0, 0, 0, 0};
+    cudaMemcpyFromSymbol(info, lora::g_status_info, sizeof(info));
+    std::fprintf(stderr, "lora_b200: bounded wait gave up (block %u, thread %u, site %u, parity %u)\n", info[0],
+                 info[1], info[2], info[3]);
+    const unsigned int zero[5] = {0, 0, 0, 0, 0};
+    cudaMemcpyToSymbol(lora::g_status, zero, sizeof(unsigned int));
+    cudaMemcpyToSymbol(lora::g_status_info, zero, sizeof(info));
+    return LORA_ERR_TIMEOUT;
+  }
+  return LORA_OK;
+}
+
+lora_status_t lora_selftest_wait_timeout(int64_t limit_ns) {
+  DeviceInfo dev;
+  lora_status_t s = device_info(dev);
+  if (s != LORA_OK) return s;
+  const uint64_t lim = uint64_t(std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 1000000000));
+  lora::selftest_wait_kernel<<<1, 32>>>(lim);
+  if ((s = launch_status()) != LORA_OK) return s;
+  return lora_get_device_status();
+}
+
+}  // extern "C"

@@ -1,6 +1,8 @@
 import os
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -8,3 +10,22 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
+
+
+@pytest.fixture(scope="session")
+def built_lib():
+    """Build the C-ABI library if it is missing or stale, return the binding."""
+    from lora_linear_layer_b200 import build as B
+    B.build(verbose=False)
+    import lora_linear_layer_b200 as L
+    L.lib()
+    return L
+
+
+@pytest.fixture(scope="session")
+def gpu(built_lib):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test selected but no CUDA device is visible")
+    torch.cuda.set_device(0)
+    return built_lib

@@ -1,0 +1,127 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/lora.h declares, and validates arguments on the host exactly as the
+entry points do (no CUDA call is made on these paths)."""
+import ctypes
+import re
+
+import pytest
+
+ALIGNED = 0x7f0000001000      # never dereferenced: validation only
+
+
+def test_library_loads_and_exports_every_header_function(built_lib):
+    L = built_lib
+    names = L.header_functions()
+    assert len(names) >= 10, names
+    so = L.lib()
+    for n in names:
+        assert hasattr(so, n), f"{n} declared in include/lora.h but not exported"
+    assert L.lora_abi_version() == 1
+
+
+def test_header_declares_the_hot_path_entry_points(built_lib):
+    names = set(built_lib.header_functions())
+    for n in ("lora_fwd", "lora_bwd", "lora_bwd_workspace_size", "lora_merge", "lora_merge_batched",
+              "lora_restore", "lora_get_device_status", "lora_check_args", "lora_status_string"):
+        assert n in names
+
+
+def test_status_strings(built_lib):
+    L = built_lib
+    for code, name in L.STATUS.items():
+        assert L.lora_status_string(code).startswith(name)
+
+
+def _ptrs(n, base=ALIGNED, step=1 << 32):
+    return [base + i * step for i in range(n)]
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,expect", [
+    (256, 512, 512, 16, "LORA_OK"),
+    (0, 512, 512, 16, "LORA_OK"),
+    (3, 8, 8, 8, "LORA_OK"),
+    (-1, 512, 512, 16, "LORA_ERR_SHAPE"),
+    (256, 0, 512, 16, "LORA_ERR_SHAPE"),
+    (256, 516, 512, 16, "LORA_ERR_SHAPE"),
+    (256, 512, 100, 16, "LORA_ERR_SHAPE"),
+    (256, 512, 512, 12, "LORA_ERR_RANK"),
+    (256, 512, 512, 0, "LORA_ERR_RANK"),
+    (256, 512, 512, 136, "LORA_ERR_RANK"),
+    (256, 512, 512, 128, "LORA_OK"),
+])
+def test_fwd_shape_and_rank_validation(built_lib, M, d_in, d_out, r, expect):
+    L = built_lib
+    assert L.STATUS[L.lora_check_args(0, _ptrs(5), M, d_in, d_out, r)] == expect
+
+
+def test_fwd_null_align_alias(built_lib):
+    L = built_lib
+    p = _ptrs(5)
+    assert L.STATUS[L.lora_check_args(0, p[:4] + [0], 8, 8, 8, 8)] == "LORA_ERR_NULL"
+    q = list(p)
+    q[2] += 8
+    assert L.STATUS[L.lora_check_args(0, q, 8, 8, 8, 8)] == "LORA_ERR_ALIGN"
+    q = list(p)
+    q[4] = q[0] + 16                       # Y inside X
+    assert L.STATUS[L.lora_check_args(0, q, 8, 8, 8, 8)] == "LORA_ERR_ALIAS"
+
+
+def test_bwd_workspace_rules(built_lib):
+    L = built_lib
+    M, d_in, d_out, r = 1000, 520, 264, 24
+    need = L.lora_bwd_workspace_size(M, d_in, d_out, r)
+    assert need > 0 and need % 256 == 0
+    assert L.lora_bwd_workspace_size(0, d_in, d_out, r) == 0
+    assert L.lora_bwd_workspace_size(M, d_in, d_out, 12) == 0          # invalid -> 0
+    # at least T and dT (bf16 [M, r_pad]) plus one fp32 partial of dA and dB
+    r_pad = 32
+    assert need >= 2 * M * r_pad * 2 + (d_in + d_out) * r_pad * 4
+    assert L.lora_bwd_workspace_size(2 * M, d_in, d_out, r) > need
+    p = _ptrs(9)
+    assert L.STATUS[L.lora_check_args(1, p, M, d_in, d_out, r, need)] == "LORA_OK"
+    assert L.STATUS[L.lora_check_args(1, p, M, d_in, d_out, r, need - 256)] == "LORA_ERR_WORKSPACE"
+    q = list(p)
+    q[8] = 0
+    assert L.STATUS[L.lora_check_args(1, q, M, d_in, d_out, r, need)] == "LORA_ERR_WORKSPACE"
+    q = list(p)
+    q[8] += 128                             # workspace must be 256-byte aligned
+    assert L.STATUS[L.lora_check_args(1, q, M, d_in, d_out, r, need)] == "LORA_ERR_ALIGN"
+    q = list(p)
+    q[5] = q[4]                             # dX aliases dY
+    assert L.STATUS[L.lora_check_args(1, q, M, d_in, d_out, r, need)] == "LORA_ERR_ALIAS"
+    q = list(p)
+    q[6] = q[8] + 256                       # dA inside the workspace
+    assert L.STATUS[L.lora_check_args(1, q, M, d_in, d_out, r, need)] == "LORA_ERR_ALIAS"
+    # M = 0 needs no workspace at all
+    q = list(p)
+    q[8] = 0
+    assert L.STATUS[L.lora_check_args(1, q, 0, d_in, d_out, r, 0)] == "LORA_OK"
+
+
+def test_merge_validation(built_lib):
+    L = built_lib
+    p = _ptrs(4)
+    assert L.STATUS[L.lora_check_args(2, p, 0, 2560, 4096, 32)] == "LORA_OK"
+    q = list(p)
+    q[3] = q[0]                             # in place is allowed
+    assert L.STATUS[L.lora_check_args(2, q, 0, 2560, 4096, 32)] == "LORA_OK"
+    q = list(p)
+    q[3] = q[0] + 64                        # partial overlap is not
+    assert L.STATUS[L.lora_check_args(2, q, 0, 2560, 4096, 32)] == "LORA_ERR_ALIAS"
+    q = list(p)
+    q[3] = q[1]                             # W_dst over A
+    assert L.STATUS[L.lora_check_args(2, q, 0, 2560, 4096, 32)] == "LORA_ERR_ALIAS"
+    assert L.STATUS[L.lora_check_args(2, p, 0, 2560, 4090, 32)] == "LORA_ERR_SHAPE"
+    assert L.STATUS[L.lora_check_args(2, p, 0, 2560, 4096, 20)] == "LORA_ERR_RANK"
+    assert L.STATUS[L.lora_check_args(2, [0] + p[1:], 0, 2560, 4096, 32)] == "LORA_ERR_NULL"
+
+
+def test_unknown_op_rejected(built_lib):
+    assert built_lib.STATUS[built_lib.lora_check_args(7, _ptrs(5), 8, 8, 8, 8)] == "LORA_ERR_SHAPE"
+
+
+def test_binding_rejects_cpu_tensors_before_any_cuda_call(built_lib):
+    import torch
+    X = torch.zeros(8, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        built_lib.lora_fwd(X, X, X[:8], X, X.clone(), 16.0)

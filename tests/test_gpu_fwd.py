@@ -1,0 +1,96 @@
+"""GPU parity of lora_fwd against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+from gpu_helpers import dev, f64, run_fwd
+from tolerance import lora_tol_check
+
+pytestmark = pytest.mark.gpu
+
+# (M, d_in, d_out, r, alpha): several tiles and ragged tails in every
+# dimension, every rank-chunk width (16/32/64) and both tile widths.
+SHAPES = [
+    (256, 512, 512, 16, 32.0),      # tiny forward workload (full check)
+    (1, 8, 8, 8, 16.0),             # smallest legal problem
+    (300, 520, 264, 8, 6.0),        # r = 8 padded to 16; scale 0.75
+    (129, 64, 136, 24, 18.0),       # r = 24 -> 32
+    (777, 1032, 1000, 40, 30.0),    # r = 40 -> 48 (64-wide chunk, partly empty)
+    (1000, 512, 2056, 64, 128.0),
+    (257, 256, 384, 128, 96.0),     # largest rank
+    (2048, 1024, 4096, 32, 64.0),   # enough tiles for 256-wide tiles
+    (640, 2048, 1544, 16, 12.0),
+]
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,alpha", SHAPES)
+def test_fwd_matches_oracle(gpu, M, d_in, d_out, r, alpha):
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=M + d_in + r)
+    Y = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+    ok, info = lora_tol_check(f64(Y), ref)
+    assert ok, info
+
+
+@pytest.mark.parametrize("shape", [WL.ATTN_PROJ, WL.MLP_UP], ids=lambda s: s.name)
+def test_fwd_full_size_sampled_rows(gpu, shape):
+    """Full-size workloads in the benchmark's launch configuration; every
+    128-row tile contributes sampled rows (plus first and last)."""
+    t = WL.make_layer_inputs(shape, seed=0)
+    Y = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], shape.alpha)
+    rows = WL.sample_rows(shape.M, seed=1, per_tile=1)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), shape.alpha, rows=rows.numpy())
+    ok, info = lora_tol_check(f64(Y.cpu()[rows]), ref)
+    assert ok, info
+    assert torch.isfinite(Y.float()).all()
+
+
+def test_fwd_zero_adapter_gives_base_and_is_bitwise_stable(gpu):
+    sh = WL.LayerShape(640, 1024, 768, 16, 32.0)
+    t = WL.make_layer_inputs(sh, seed=3)
+    zB = torch.zeros_like(t["B"])
+    zA = torch.zeros_like(t["A"])
+    Y_b0 = run_fwd(gpu, t["X"], t["W"], t["A"], zB, sh.alpha)
+    Y_a0 = run_fwd(gpu, t["X"], t["W"], zA, t["B"], sh.alpha)
+    # either factor zero => the adapter adds exact zeros to the same base sum
+    assert torch.equal(Y_b0, Y_a0)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), np.zeros((768, 16)), sh.alpha)
+    ok, info = lora_tol_check(f64(Y_b0), ref)
+    assert ok, info
+
+
+def test_fwd_deterministic(gpu):
+    sh = WL.LayerShape(1024, 1024, 2048, 32, 64.0)
+    t = WL.make_layer_inputs(sh, seed=9)
+    Y1 = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], sh.alpha)
+    Y2 = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], sh.alpha)
+    assert torch.equal(Y1, Y2)
+
+
+def test_merged_forward_equals_unmerged(gpu):
+    """X W'^T with W' = merge(W, A, B) matches the unmerged forward."""
+    sh = WL.LayerShape(512, 1024, 1024, 16, 32.0)
+    t = WL.make_layer_inputs(sh, seed=4)
+    Wd, Ad, Bd = dev(t["W"]), dev(t["A"]), dev(t["B"])
+    Wm = torch.empty_like(Wd)
+    gpu.lora_merge(Wd, Ad, Bd, Wm, sh.alpha)
+    Y_unmerged = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], sh.alpha)
+    Y_merged = run_fwd(gpu, t["X"], Wm.cpu(), t["A"], torch.zeros_like(t["B"]), sh.alpha)
+    ok, info = lora_tol_check(f64(Y_merged), f64(Y_unmerged))
+    assert ok, info
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), sh.alpha)
+    ok, info = lora_tol_check(f64(Y_merged), ref)
+    assert ok, info
+
+
+def test_fwd_empty_batch_is_noop(gpu):
+    X = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.ones((64, 64), dtype=torch.bfloat16, device="cuda")
+    A = torch.ones((16, 64), dtype=torch.bfloat16, device="cuda")
+    B = torch.ones((64, 16), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    gpu.lora_fwd(X, W, A, B, Y, 32.0)
+    assert gpu.lora_get_device_status() == 0

@@ -1,0 +1,117 @@
+"""GPU parity of lora_merge / lora_merge_batched / lora_restore against the
+oracle, and the restore-from-pristine bit-identity over refresh cycles."""
+import hashlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+from gpu_helpers import dev, f64
+from tolerance import merge_tol_check
+
+pytestmark = pytest.mark.gpu
+
+
+def _merge_check(t, W_out, r, alpha):
+    W, A, B = f64(t["W"]), f64(t["A"]), f64(t["B"])
+    exact = O.lora_merge(W, A, B, alpha)
+    ok, info = merge_tol_check(f64(W_out), exact, W, A, B, alpha / r)
+    assert ok, info
+    return info
+
+
+@pytest.mark.parametrize("d_out,d_in,r", [(96, 80, 32), (4096, 2560, 32), (1000, 520, 24), (2560, 9728, 32),
+                                          (136, 64, 8), (520, 1032, 64), (264, 384, 128)])
+def test_merge_matches_oracle(gpu, d_out, d_in, r):
+    alpha = 2.0 * r
+    t = WL.make_merge_inputs(d_out, d_in, r, seed=d_out + d_in)
+    Wd, Ad, Bd = dev(t["W"]), dev(t["A"]), dev(t["B"])
+    out = torch.full_like(Wd, float("nan"))
+    gpu.lora_merge(Wd, Ad, Bd, out, alpha)
+    assert gpu.lora_get_device_status() == 0
+    info = _merge_check(t, out, r, alpha)
+    assert info["max_ulps_noncancel"] <= 1.0 and info["frac_noncancel"] > 0.99, info
+    assert torch.equal(Wd.cpu(), t["W"])          # the pristine source is untouched
+
+
+def test_merge_in_place_equals_out_of_place(gpu):
+    t = WL.make_merge_inputs(1024, 2560, 32, seed=1)
+    Wd, Ad, Bd = dev(t["W"]), dev(t["A"]), dev(t["B"])
+    out = torch.empty_like(Wd)
+    gpu.lora_merge(Wd, Ad, Bd, out, 64.0)
+    inplace = Wd.clone()
+    gpu.lora_merge(inplace, Ad, Bd, inplace, 64.0)
+    assert torch.equal(out, inplace)
+
+
+def test_merge_zero_B_is_bitwise_identity(gpu):
+    t = WL.make_merge_inputs(1024, 2560, 32, seed=2)
+    Wd, Ad = dev(t["W"]), dev(t["A"])
+    out = torch.empty_like(Wd)
+    gpu.lora_merge(Wd, Ad, torch.zeros((1024, 32), dtype=torch.bfloat16, device="cuda"), out, 64.0)
+    assert torch.equal(out, Wd)
+
+
+def test_restore_is_bit_copy(gpu):
+    t = WL.make_merge_inputs(1000, 520, 24, seed=3)
+    Wd = dev(t["W"])
+    dst = torch.full_like(Wd, 3.0)
+    gpu.lora_restore(Wd, dst)
+    assert torch.equal(dst, Wd)
+    odd_src = Wd.flatten()[: Wd.numel() - 3 * 8].contiguous()     # length not a multiple of 8? keep aligned
+    odd_dst = torch.zeros_like(odd_src)
+    gpu.lora_restore(odd_src, odd_dst)
+    assert torch.equal(odd_src, odd_dst)
+
+
+def _sha(t):
+    return hashlib.sha256(t.cpu().view(torch.int16).numpy().tobytes()).hexdigest()
+
+
+def test_batched_merge_matches_single_and_restore_cycles_bit_identical(gpu):
+    """Two layers of the 7-target merge workload: batched == per-matrix merges
+    bitwise; every matrix within the merge bound; ten perturb + restore +
+    merge refreshes leave the pristine copy bit-identical and make the merged
+    state a function of (pristine, A, B) only."""
+    r, alpha = WL.MERGE_R, WL.MERGE_ALPHA
+    shapes = WL.merge_shapes(layers=2)
+    mats = [WL.make_merge_inputs(s["d_out"], s["d_in"], r, seed=100 + i) for i, s in enumerate(shapes)]
+    pristine = [dev(m["W"]) for m in mats]
+    Ad = [dev(m["A"]) for m in mats]
+    Bd = [dev(m["B"]) for m in mats]
+    h0 = [_sha(p) for p in pristine]
+    W_inf = [p.clone() for p in pristine]
+
+    gpu.lora_merge_batched(list(zip(pristine, Ad, Bd, W_inf)), r, alpha)
+    assert gpu.lora_get_device_status() == 0
+    for i, m in enumerate(mats):
+        single = torch.empty_like(pristine[i])
+        gpu.lora_merge(pristine[i], Ad[i], Bd[i], single, alpha)
+        assert torch.equal(single, W_inf[i])
+        _merge_check(m, W_inf[i], r, alpha)
+
+    first_state = None
+    for cycle in range(10):
+        A_new, B_new = [], []
+        for i, m in enumerate(mats):
+            a, b = WL.perturb_adapter(m["A"], m["B"], cycle)
+            A_new.append(dev(a))
+            B_new.append(dev(b))
+        for i in range(len(mats)):
+            gpu.lora_restore(pristine[i], W_inf[i])
+            assert torch.equal(W_inf[i], pristine[i])
+        gpu.lora_merge_batched(list(zip(pristine, A_new, B_new, W_inf)), r, alpha)
+        again = [torch.empty_like(p) for p in pristine]
+        gpu.lora_merge_batched(list(zip(pristine, A_new, B_new, again)), r, alpha)
+        for x, y in zip(W_inf, again):
+            assert torch.equal(x, y)
+        if cycle == 0:
+            first_state = [w.clone() for w in W_inf]
+    assert [_sha(p) for p in pristine] == h0
+    # re-merging the cycle-0 adapter from pristine reproduces that state exactly
+    for i, m in enumerate(mats):
+        a, b = WL.perturb_adapter(m["A"], m["B"], 0)
+        gpu.lora_merge(pristine[i], dev(a), dev(b), W_inf[i], alpha)
+        assert torch.equal(W_inf[i], first_state[i])

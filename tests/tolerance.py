@@ -8,7 +8,8 @@
   plus the forward error bound of an fp32 accumulation of the r-term rank
   product and the add:  (r + 2) * 2**-24 * (|W| + |s| * (|B| @ |A|)).
   That second term only matters where W and s*B@A cancel to a value whose
-  own bf16 ULP is below the fp32 rounding of the summands.
+  own bf16 ULP is below the fp32 rounding of the summands; everywhere else
+  (|exact| >= (r+2) 2^-14 (|W| + |s| |B| @ |A|)) one ULP is required.
 """
 from __future__ import annotations
 
@@ -48,6 +49,12 @@ def merge_tol_check(w, w_exact, W_src, A, B, scale: float):
     bound = ulp_bf16(w_exact) + (r + 2) * 2.0 ** -24 * acc_mag
     err = np.abs(w - w_exact)
     bad = ~(err <= bound)
+    ulps = err / ulp_bf16(w_exact)
+    # where |exact| >= (r+2) 2^-14 acc_mag the fp32 accumulation error is at
+    # most half a bf16 ULP of the result, so one ULP must hold there
+    noncancel = np.abs(w_exact) >= (r + 2) * 2.0 ** -14 * acc_mag
     info = dict(n=int(w.size), n_bad=int(bad.sum()), max_err=float(err.max()) if err.size else 0.0,
-                max_err_in_ulps=float((err / ulp_bf16(w_exact)).max()) if err.size else 0.0)
+                max_err_in_ulps=float(ulps.max()) if err.size else 0.0,
+                max_ulps_noncancel=float(ulps[noncancel].max()) if noncancel.any() else 0.0,
+                frac_noncancel=float(noncancel.mean()) if err.size else 1.0)
     return not bad.any(), info
