@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the fused LoRA layer hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic
+input: lora_fwd (Y), lora_bwd (dX, dA, dB; T recomputed) and lora_merge
+(W' = W + s B A) on the attention-projection workload X[8192, 4096],
+W[4096, 4096], r = 16, alpha = 32.  With N > 1 GPUs every rank runs the
+same step on its own batch (data parallel along M, weak scaling) and the
+adapter gradients dA, dB are summed across ranks with one NCCL all-reduce.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Metric: TFLOP/s of algorithmic work
+(counted below; no recompute, no padding) over device time, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+_ROOT = os.path.dirname(os.path.abspath(__file__))
+if _ROOT not in sys.path:
+    sys.path.insert(0, _ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "fused LoRA fwd/bwd TFLOP/s (bf16) and % of B200 dense peak; µs/call"
+UNIT = "TFLOP/s"
+WORKLOAD = WL.ATTN_PROJ
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
+                  "lora_linear_layer_b200/csrc/common.cuh")
+LAUNCHES_PER_STEP = 8   # fwd 1; bwd: T, dX, dB, dA, 2 reductions; merge 1
+
+
+# ------------------------------------------------------ algorithmic work ----
+
+def flops_fwd(M, d_in, d_out, r):
+    return 2.0 * M * (d_in * d_out + r * d_in + r * d_out)
+
+
+def flops_bwd(M, d_in, d_out, r):
+    # dX = dY W + dT A; dT = s dY B; dB = s dY^T T; dA = dT^T X (T recompute not counted)
+    return 2.0 * M * (d_out * d_in + r * d_in) + 2.0 * M * d_out * r * 2 + 2.0 * M * r * d_in
+
+
+def flops_merge(d_in, d_out, r):
+    return 2.0 * r * d_out * d_in
+
+
+def step_flops(sh):
+    return (flops_fwd(sh.M, sh.d_in, sh.d_out, sh.r) + flops_bwd(sh.M, sh.d_in, sh.d_out, sh.r)
+            + flops_merge(sh.d_in, sh.d_out, sh.r))
+
+
+# ---------------------------------------------------------------- peaks ----
+
+def load_peaks():
+    p = os.path.join(_ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_src_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(_ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, src_hash):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(_ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                    and parts[2] == src_hash:
+                return float(parts[3])
+    return None
+
+
+# --------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ reference ----
+
+def oracle_step_sample(t, sh, rows):
+    """One sampled step of the fp64 oracle: forward and backward on the first
+    `rows` rows of the batch, merge of the full weight."""
+    import oracle as O
+    X = t["X"][:rows]
+    dY = t["dY"][:rows]
+    f = lambda x: O.bf16_bits_to_f64(WL.bf16_bits(x))  # noqa: E731
+    Xf, Wf, Af, Bf, dYf = f(X), f(t["W"]), f(t["A"]), f(t["B"]), f(dY)
+    O.lora_forward(Xf, Wf, Af, Bf, sh.alpha)
+    O.lora_backward(Xf, Wf, Af, Bf, dYf, sh.alpha)
+    O.lora_merge(Wf, Af, Bf, sh.alpha)
+    return (flops_fwd(rows, sh.d_in, sh.d_out, sh.r) + flops_bwd(rows, sh.d_in, sh.d_out, sh.r)
+            + flops_merge(sh.d_in, sh.d_out, sh.r))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(sh, budget_s=12.0, rows=512):
+    """Time the oracle as it stands on a bounded sample of the workload."""
+    t = WL.make_layer_inputs(WL.LayerShape(rows, sh.d_in, sh.d_out, sh.r, sh.alpha), seed=0, with_dy=True)
+    flops, n = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        flops += oracle_step_sample(t, sh, rows)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} sampled steps: fwd+bwd on {rows} of {sh.M} rows, merge of the full "
+                      f"{sh.d_out}x{sh.d_in} weight, fp64 numpy/BLAS; {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sh = WORKLOAD
+    rows = 512
+    t = WL.make_layer_inputs(WL.LayerShape(rows, sh.d_in, sh.d_out, sh.r, sh.alpha), seed=0, with_dy=True)
+    for _ in range(max(args.warmup, 0)):
+        oracle_step_sample(t, sh, rows)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        flops += oracle_step_sample(t, sh, rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = flops / total / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": sh.name, "M": sh.M, "d_in": sh.d_in, "d_out": sh.d_out, "r": sh.r,
+                   "alpha": sh.alpha, "sample_rows": rows, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: fp64 oracle fwd+bwd on {rows} of {sh.M} rows + full merge"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours ----
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import lora_linear_layer_b200 as L
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    L.lib()
+
+    sh = WORKLOAD
+    M, d_in, d_out, r, alpha = sh.M, sh.d_in, sh.d_out, sh.r, sh.alpha
+    host = WL.make_layer_inputs(sh, seed=rank, with_dy=True)
+    X, W, A, B, dY = (host[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty((M, d_in), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((r, d_in), dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty((d_out, r), dtype=torch.bfloat16, device="cuda")
+    Wm = torch.empty_like(W)
+    ws = torch.empty(L.lora_bwd_workspace_size(M, d_in, d_out, r), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev_f0=None, ev_f1=None):
+        if ev_f0 is not None:
+            ev_f0.record(stream)
+        L.lora_fwd(X, W, A, B, Y, alpha, stream)
+        if ev_f1 is not None:
+            ev_f1.record(stream)
+        L.lora_bwd(X, W, A, B, dY, dX, dA, dB, alpha, ws, stream)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+        L.lora_merge(W, A, B, Wm, alpha, stream)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    if L.lora_get_device_status() != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(K):
+        flush.zero_()                       # evict L2 (outside the timed pairs)
+        s0, s1, f0, f1 = ev[i]
+        s0.record(stream)
+        step(f0, f1)
+        s1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    if L.lora_get_device_status() != 0:
+        raise SystemExit("device status not OK after the timed region")
+    step_ms = [s0.elapsed_time(s1) for (s0, s1, _, _) in ev]
+    fwd_ms = [f0.elapsed_time(f1) for (_, _, f0, f1) in ev]
+    total_ms = sum(step_ms)
+    fwd_avg_ms = sum(fwd_ms) / K
+    t_local = torch.tensor([total_ms, fwd_avg_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    total_ms, fwd_avg_ms = float(t_local[0]), float(t_local[1])
+
+    # ---------------- end to end through the C ABI with host buffers -------
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: host[k].pin_memory() for k in ("X", "W", "A", "B", "dY")}
+        out_dA = torch.empty_like(dA, device="cpu").pin_memory()
+        out_dB = torch.empty_like(dB, device="cpu").pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = out_dA.numel() * 2 + out_dB.numel() * 2
+        Ke = max(3, min(K, args.e2e_steps))
+
+        def e2e_step():
+            X.copy_(pin["X"], non_blocking=True)
+            W.copy_(pin["W"], non_blocking=True)
+            A.copy_(pin["A"], non_blocking=True)
+            B.copy_(pin["B"], non_blocking=True)
+            dY.copy_(pin["dY"], non_blocking=True)
+            step()
+            out_dA.copy_(dA, non_blocking=True)
+            out_dB.copy_(dB, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": step_flops(sh) * Ke * world / (float(e_ms[0]) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": Ke,
+               "what": "every step copies X, W, A, B, dY from pinned host memory and reads dA, dB back"}
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    value = step_flops(sh) * K * world / (total_ms * 1e-3) / 1e12
+    fwd_flops = flops_fwd(M, d_in, d_out, r)
+    achieved = fwd_flops / (fwd_avg_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    src_hash = kernel_src_hash()
+    traffic = recorded_traffic("fused_lora_kernel_fwd", sh.name, src_hash)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded normal inputs, bf16)",
+        "config": {"workload": sh.name, "M": M, "d_in": d_in, "d_out": d_out, "r": r, "alpha": alpha,
+                   "global_batch_tokens": M * world, "step": "lora_fwd + lora_bwd + lora_merge",
+                   "l2": "flushed between steps (256 MB write outside the timed pairs); inputs > L2",
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU"},
+        "breakdown": {"fwd_us": 1e3 * fwd_avg_ms, "fwd_tflops": achieved,
+                      "rest_of_step_us": 1e3 * (total_ms / K - fwd_avg_ms)},
+        "roofline": {"kernel": "fused_lora_kernel (forward)", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "peak_burst": float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+                     "algorithmic_flops_per_launch": fwd_flops, "src_hash": src_hash},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(sh, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

