@@ -111,6 +111,33 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward without a workspace argument (the pages describe no such entry
+ * point; it is a service of this library, not part of the method).
+ *
+ * Same arguments, results and rules as lora_bwd, minus `workspace` and
+ * `workspace_bytes`.  It is for callers that cannot call cudaMalloc, such
+ * as a plugin whose host program owns all device memory through its own
+ * pool, or a service loop that must not allocate after start-up because
+ * cudaMalloc can wait for the device to go idle and can fail under memory
+ * pressure.  Instead of a caller workspace it uses a fixed 32 MiB scratch
+ * array that the library reserves in device global memory on every GPU
+ * that loads it, for the life of the process.
+ *  - Shapes whose lora_bwd_workspace_size(...) exceeds 32 MiB are refused
+ *    with LORA_ERR_WORKSPACE (and a message on stderr) before any launch.
+ *  - The first call on each device looks up the array's device address
+ *    (with that device current) and keeps it; make that first call before
+ *    any stream capture begins.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    nothing in it needs to start at zero.  Calls whose work can overlap on
+ *    the GPU (e.g. on two streams) race on it: keep them on one stream.
+ *  - Allocates no device memory.
+ */
+lora_status_t lora_bwd_noalloc(const void* X, const void* W, const void* A, const void* B,
+                               const void* dY, void* dX, void* dA, void* dB,
+                               int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                               void* stream);
+
+/*
  * Merge: W_dst[d_out, d_in] = bf16_rne(W_src + s * (B A)), the rank-r
  * product accumulated in fp32 and rounded once.  W_src is the pristine base
  * (restore + merge in one pass) or W_dst itself (in place).

@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.lora_bwd_workspace_size.argtypes = [i64, i64, i64, i32]
         L.lora_bwd.restype = ctypes.c_int
         L.lora_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, vp]
+        L.lora_bwd_noalloc.restype = ctypes.c_int
+        L.lora_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
         L.lora_merge.restype = ctypes.c_int
         L.lora_merge.argtypes = [vp, vp, vp, vp, i64, i64, i32, f32, vp]
         L.lora_merge_batched.restype = ctypes.c_int
@@ -159,6 +161,22 @@ def lora_bwd(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, stream=None) -
     code = lib().lora_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
                           M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, _stream(stream))
     _raise(code, "lora_bwd")
+
+
+def lora_bwd_noalloc(X, W, A, B, dY, dX, dA, dB, alpha: float, stream=None) -> None:
+    """lora_bwd for callers that cannot allocate device memory: the scratch
+    is the library's own fixed 32 MiB per-device array (see include/lora.h).
+    Calls that may overlap on the GPU share that array; keep them on one
+    stream."""
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r)), (dY, "dY", (M, d_out)), (dX, "dX", (M, d_in)),
+                    (dA, "dA", (r, d_in)), (dB, "dB", (d_out, r))):
+        _check_tensor(t, n, s)
+    code = lib().lora_bwd_noalloc(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
+                                  M, d_in, d_out, r, float(alpha), _stream(stream))
+    _raise(code, "lora_bwd_noalloc")
 
 
 def lora_merge(W_src, A, B, W_dst, alpha: float, stream=None) -> None:

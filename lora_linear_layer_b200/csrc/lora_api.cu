@@ -650,3 +650,86 @@ lora_status_t lora_selftest_wait_timeout(int64_t limit_ns) {
 }
 
 }  // extern "C"
+
+// ====================================================== no-alloc backward ====
+//
+// lora_bwd_noalloc: the backward for callers that cannot call cudaMalloc.
+//
+// lora_bwd needs device scratch (T, dT and the split-M partial sums) and
+// asks the caller for it.  Some callers have no way to provide it: a plugin
+// running inside a host program that owns every device allocation through
+// its own pool, or a service loop that must not allocate once it has
+// started (cudaMalloc can block until the device is idle, and can fail
+// when memory is tight, at a point where the caller cannot recover).  This
+// entry point serves them with scratch that the library reserves itself:
+// a fixed-size array in device global memory, part of the library's GPU
+// module.  It is reserved on every GPU that loads the library and stays
+// there until the process exits.
+//
+// The array is a file-scope __device__ symbol, so host code cannot use its
+// name as a device address (on the host the name refers to a host-side
+// stand-in).  The first call on each device, with that device current,
+// looks the real address up with cudaGetSymbolAddress, checks the result,
+// and keeps it for later calls on that device; that first call should be
+// made before any stream capture begins.  The kernels then receive that
+// address exactly as they would receive a caller's workspace.
+//
+// All calls share the one array, and it keeps whatever the previous call
+// left in it.  Nothing in it needs to start at zero: each call writes every
+// scratch byte before reading it.  Two calls whose work can overlap on the
+// GPU (for example on two different streams) use the same bytes at the same
+// time and corrupt each other's results; order them on one stream.
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_bwd_noalloc_scratch on the current device (looked up
+// once per device).
+lora_status_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      std::fprintf(stderr, "lora_bwd_noalloc: cudaGetSymbolAddress failed on device %d: %s\n", dev,
+                   cudaGetErrorString(e));
+      return LORA_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return LORA_OK;
+}
+}  // namespace
+
+extern "C" lora_status_t lora_bwd_noalloc(const void* X, const void* W, const void* A, const void* B,
+                                          const void* dY, void* dX, void* dA, void* dB, int64_t M,
+                                          int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
+  lora_status_t s = check_sizes(M, d_in, d_out, r);
+  if (s != LORA_OK) return s;
+  const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
+  if (need > kNoAllocScratchBytes) {
+    std::fprintf(stderr,
+                 "lora_bwd_noalloc: M=%lld d_in=%lld d_out=%lld r=%d needs %zu bytes of scratch, more than the "
+                 "fixed %zu bytes this entry point has; call lora_bwd with a workspace instead\n",
+                 (long long)M, (long long)d_in, (long long)d_out, int(r), need, kNoAllocScratchBytes);
+    return LORA_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if (need > 0) {
+    DeviceInfo dev;
+    if ((s = device_info(dev)) != LORA_OK) return s;
+    if ((s = noalloc_scratch_address(&scratch)) != LORA_OK) return s;
+  }
+  return lora_bwd(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+                  stream);
+}
