@@ -24,13 +24,16 @@ enum WaitSite : uint32_t {
 // global timer, and gives up (returning false) once `limit_ns` has passed or
 // another role of the CTA has already given up.  On the first give-up it
 // raises the CTA abort flag and records the failure in the status word.
+// `cluster_scope` makes the wait an acquire at cluster scope, for barriers
+// that other CTAs of the cluster arrive on.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             uint64_t limit_ns, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                             uint64_t limit_ns, uint32_t site, bool cluster_scope = false) {
+  auto probe = [&]() { return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (probe()) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (probe()) return true;
     if ((++spins & 63u) == 0u) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > limit_ns) {
@@ -52,9 +55,9 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 // instructions: lane 0 polls, the verdict is broadcast, and __syncwarp
 // orders the other lanes after lane 0's observation of the barrier.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                                  uint64_t limit_ns, uint32_t site) {
+                                                  uint64_t limit_ns, uint32_t site, bool cluster_scope = false) {
   int ok = 1;
-  if ((threadIdx.x & 31u) == 0u) ok = wait_bounded(bar, parity, abort_flag, limit_ns, site) ? 1 : 0;
+  if ((threadIdx.x & 31u) == 0u) ok = wait_bounded(bar, parity, abort_flag, limit_ns, site, cluster_scope) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   __syncwarp();
   return ok != 0;

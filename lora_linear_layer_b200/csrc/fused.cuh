@@ -4,34 +4,45 @@
 //   forward  (MN = false): P = X[M,d_in], Q = W[d_out,d_in], U = A[r,d_in],
 //                          V = B[d_out,r]; all operands K-major.
 //                          OUT = Y = X W^T + s (X A^T) B^T
-//   dX       (MN = true):  P = dY[M,d_out], Q(n,k) = W[k,n], U(j,k) = B[k,j],
-//                          V(n,j) = A[j,n]; Q, U, V are read MN-major.
+//   dX       (MN = true):  P = dY[M,d_out], Q(n,k) = W[k,n] and V(n,j) = A[j,n]
+//                          read MN-major, U = B^T[r,d_out] (a transposed copy
+//                          of B, K-major).
 //                          OUT = dX = dY W + (s dY B) A, and the bf16 dT = s dY B
 //                          is also written out (for dA).
 // (fastaf 0.1.0, "FWD kernel speedup": base product plus the down- and
 // up-projections, scale and add; "BWD kernel speedup": the dX kernel.)
 //
-// Per 128 x BN output tile:
+// Per output tile of (128 * CG) x BN:
 //   * the K loop streams P, Q (and, on the first tile of an M block, U)
-//     through a TMA -> shared-memory ring; one thread issues
-//     tcgen05.mma for the base product into a TMEM accumulator and, on that
-//     first tile, the N = r product T = P U^T into a second TMEM region;
+//     through a TMA -> shared-memory ring; one thread issues tcgen05.mma
+//     for the base product into a TMEM accumulator and, on that first tile,
+//     the N = r product T = P U^T into a second TMEM region;
 //   * four epilogue warps drain T, scale it by s in fp32, round to bf16 and
 //     write it into shared memory in the UMMA K-major swizzled layout (it
 //     never goes to global memory in the forward);
 //   * one more MMA pass (K = r) accumulates (sT) V^T onto the base
 //     accumulator; the epilogue rounds once to bf16 and stores.
 // T is kept in shared memory and reused for every further tile of the same
-// M block the CTA processes (tiles are scheduled so a CTA sweeps N within
-// an M block).  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)...).
+// M block the CTA processes.  Warp roles: warp 0 = TMA producer, warp 1 =
+// MMA issuer and TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes
+// 32*(w%4)...).
+//
+// CG = 2 runs each tile on a CTA pair (a cluster of two, cta_group::2):
+// each CTA holds its own 128 rows of P and half of the Q/U/V rows, the even
+// CTA issues every MMA (M = 256) for both, and each CTA keeps its 128 rows
+// of every accumulator in its own TMEM.  The pair's TMA loads count their
+// bytes on the even CTA's barriers; tcgen05.commit arrives on both CTAs'
+// barriers; the odd CTA's epilogue arrives on the even CTA's barriers
+// through shared::cluster addresses.  No load is multicast.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
 namespace lora {
 
-constexpr int kBM = 128;          // tile rows (UMMA M)
+constexpr int kBM = 128;          // rows per CTA (UMMA M per CTA)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr int kFusedThreads = 192;
 
@@ -43,21 +54,23 @@ struct FusedArgs {
   float scale;              // s = alpha / r
   __nv_bfloat16* out;       // [M, N] row-major, ld = N
   __nv_bfloat16* t_out;     // optional [M, r_pad] bf16 copy of s*T (dT), or null
-  int32_t num_m, num_n;     // tile counts
+  int32_t num_m, num_n;     // tile counts (M tiles of 128 * CG rows)
   int32_t band_w, n_bands;  // column bands of the schedule
+  int32_t run_l;            // 0: contiguous ranges; L > 0: runs of L N-tiles dealt round-robin
   uint64_t wait_limit_ns;
 };
 
-// Byte sizes / offsets of the shared-memory carve-up (host and device).
+// Byte sizes / offsets of one CTA's shared-memory carve-up (host and device).
 struct FusedLayout {
   uint32_t p_bytes, q_bytes, u_bytes, stage_bytes, v_bytes, st_bytes;
   uint32_t off_v, off_st, off_bar, total;
-  __host__ __device__ FusedLayout(int BN, bool mn, int rcw, int r_pad, int n_rchunks, int stages) {
+  __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages) {
+    const int bnc = BN / CG;            // Q / V rows held by this CTA
     p_bytes = kBM * kBK * 2;
-    q_bytes = BN * kBK * 2;
-    u_bytes = mn ? uint32_t(n_rchunks * rcw * 128) : uint32_t(r_pad * 128);
+    q_bytes = uint32_t(bnc * kBK * 2);
+    u_bytes = uint32_t((r_pad / CG) * 128);
     stage_bytes = p_bytes + q_bytes + u_bytes;
-    v_bytes = mn ? uint32_t((BN / 64) * r_pad * 128) : uint32_t(n_rchunks * BN * rcw * 2);
+    v_bytes = mn ? uint32_t((bnc / 64) * r_pad * 128) : uint32_t(n_rchunks * bnc * rcw * 2);
     st_bytes = uint32_t(n_rchunks * kBM * rcw * 2);
     off_v = stage_bytes * stages;
     off_st = off_v + v_bytes;
@@ -66,18 +79,42 @@ struct FusedLayout {
   }
 };
 
-// Tile schedule: the N tiles are grouped into column bands; the tiles of a
-// band are ordered M-major (N fastest) and split into gridDim.x contiguous
-// ranges.  A CTA therefore sweeps N inside one or two M blocks per band,
-// which lets it keep T of an M block on chip, while all CTAs work in the
-// same band (bounded L2 footprint).
+// Tile schedule over clusters (one cluster = CG CTAs = one tile at a time).
+//  run_l == 0: the N tiles are grouped into column bands; the tiles of a band
+//    are ordered M-major (N fastest) and split into G contiguous ranges, so a
+//    cluster sweeps N inside one or two M blocks per band.
+//  run_l > 0: "runs" of run_l consecutive N tiles of one M block, ordered
+//    M-major, are dealt round-robin to the clusters: the tiles in flight at
+//    any time cover only ~G*run_l/num_n M blocks (compact L2 footprint),
+//    and T is computed once per run.
 struct TileSched {
-  int num_m, num_n, band_w, n_bands, G, c;
+  int num_m, num_n, band_w, n_bands, run_l, G, c;
   int band, t, t_end, band_n0, w;
-  __device__ TileSched(const FusedArgs& a)
-      : num_m(a.num_m), num_n(a.num_n), band_w(a.band_w), n_bands(a.n_bands), G(gridDim.x),
-        c(blockIdx.x), band(-1), t(0), t_end(0), band_n0(0), w(1) {}
+  int runs_per_m, run, run_end, run_pos, run_len, run_m, run_n0;
+  __device__ TileSched(const FusedArgs& a, int G_, int c_)
+      : num_m(a.num_m), num_n(a.num_n), band_w(a.band_w), n_bands(a.n_bands), run_l(a.run_l), G(G_), c(c_),
+        band(-1), t(0), t_end(0), band_n0(0), w(1), runs_per_m(1), run(0), run_end(0), run_pos(0), run_len(0),
+        run_m(0), run_n0(0) {
+    if (run_l > 0) {
+      runs_per_m = (num_n + run_l - 1) / run_l;
+      run = c - G;
+      run_end = num_m * runs_per_m;
+    }
+  }
   __device__ bool next(int& m, int& n) {
+    if (run_l > 0) {
+      if (run_pos >= run_len) {
+        run += G;
+        if (run >= run_end) return false;
+        run_m = run / runs_per_m;
+        run_n0 = (run % runs_per_m) * run_l;
+        run_len = imin(run_l, num_n - run_n0);
+        run_pos = 0;
+      }
+      m = run_m;
+      n = run_n0 + run_pos++;
+      return true;
+    }
     while (t >= t_end) {
       if (++band >= n_bands) return false;
       band_n0 = band * band_w;
@@ -94,25 +131,75 @@ struct TileSched {
   }
 };
 
-template <int BN, bool MN, int RCW>
+// PTX forms by CTA-group size.
+template <int CG>
+struct Group;
+
+template <>
+struct Group<1> {
+  static __device__ __forceinline__ void alloc(uint32_t slot, uint32_t n) {
+    tmem_alloc(slot, n);
+    tmem_relinquish();
+  }
+  static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc(t, n); }
+  static __device__ __forceinline__ void load(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1) {
+    tma_load_2d(dst, tm, bar, c0, c1);
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_bf16(d, a, b, id, acc);
+  }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { umma_commit(bar); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { umma_commit(bar); }
+  static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return bar; }
+  static __device__ __forceinline__ void arrive_leader(uint32_t bar) { mbar_arrive(bar); }
+  static __device__ __forceinline__ void cluster_sync() {}
+};
+
+template <>
+struct Group<2> {
+  static __device__ __forceinline__ void alloc(uint32_t slot, uint32_t n) {
+    tmem_alloc_pair(slot, n);
+    tmem_relinquish_pair();
+  }
+  static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc_pair(t, n); }
+  static __device__ __forceinline__ void load(uint32_t dst, const CUtensorMap* tm, uint32_t bar_leader, int c0,
+                                              int c1) {
+    tma_load_2d_pair(dst, tm, bar_leader, c0, c1);
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_bf16_pair(d, a, b, id, acc);
+  }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { umma_commit_pair_mc(bar, uint16_t(3)); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { umma_commit_pair(bar); }
+  static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return mapa_shared(bar, 0); }
+  static __device__ __forceinline__ void arrive_leader(uint32_t bar) { mbar_arrive_cluster(mapa_shared(bar, 0)); }
+  static __device__ __forceinline__ void cluster_sync() { cluster_barrier_sync(); }
+};
+
+template <int BN, bool MN, int RCW, int CG>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_lora_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
                       const FusedArgs a) {
   static_assert(BN == 128 || BN == 256, "BN");
+  static_assert(CG == 1 || CG == 2, "CG");
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
+  using G = Group<CG>;
+  constexpr int BNC = BN / CG;          // Q / V rows held by this CTA
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
   constexpr uint32_t kRSpan = RCW * 2;  // bytes per swizzled rank row
+  constexpr bool kClusterScope = CG > 1;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (sbase - raw);
 
-  const FusedLayout L(BN, MN, RCW, a.r_pad, a.n_rchunks, a.stages);
+  const FusedLayout L(BN, CG, MN, RCW, a.r_pad, a.n_rchunks, a.stages);
   const int S = a.stages;
   const uint32_t bar0 = sbase + L.off_bar;
-  // barrier map (8 bytes each)
+  // barrier map (8 bytes each); full / vfull / accempty / stfull / drain
+  // are used on the even CTA only
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
   const uint32_t vfull = bar0 + 8u * (2 * S + 0);
@@ -127,6 +214,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG > 1 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -137,10 +226,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     mbar_init(vempty, 1);
     mbar_init(accfull0, 1);
     mbar_init(accfull0 + 8, 1);
-    mbar_init(accempty0, 4);
-    mbar_init(accempty0 + 8, 4);
+    mbar_init(accempty0, 4 * CG);
+    mbar_init(accempty0 + 8, 4 * CG);
     mbar_init(tfull, 1);
-    mbar_init(stfull, 4);
+    mbar_init(stfull, 4 * CG);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -151,12 +240,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     tma_prefetch_desc(&tmU);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), 512);
-    tmem_relinquish();
-  }
+  if (warp == 1) G::alloc(smem_addr(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
+  G::cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -165,11 +252,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const bool borrow = (2 * BN + a.r_pad) > 512;
   const int nk = (a.K + kBK - 1) / kBK;
   const uint64_t lim = a.wait_limit_ns;
+  const int n_clusters = int(gridDim.x) / CG;
+  const int cluster_id = int(blockIdx.x) / CG;
+  const int u_rows = a.r_pad / CG;        // U rows held by this CTA
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
     if (lane == 0) {
-      TileSched sch(a);
+      TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
       uint32_t phase = 0, vcount = 0;
       bool ok = true;
@@ -177,55 +267,53 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const bool ttile = (m != prev_m);
         prev_m = m;
         const uint32_t bytes = L.p_bytes + L.q_bytes + (ttile ? L.u_bytes : 0u);
+        const int row0 = m * (kBM * CG) + int(rank) * kBM;
+        const int qrow0 = n * BN + int(rank) * BNC;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, lim, SITE_EMPTY)) { ok = false; break; }
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, lim, SITE_EMPTY, kClusterScope)) {
+            ok = false;
+            break;
+          }
           const uint32_t st = sbase + uint32_t(stage) * L.stage_bytes;
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, bytes);
+          const uint32_t fb = G::leader_addr(full_bar(stage));
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), bytes * CG);
           const int k0 = kb * kBK;
-          tma_load_2d(st, &tmP, fb, k0, m * kBM);
+          G::load(st, &tmP, fb, k0, row0);
           if (!MN) {
-            tma_load_2d(st + L.p_bytes, &tmQ, fb, k0, n * BN);
+            G::load(st + L.p_bytes, &tmQ, fb, k0, qrow0);
           } else {
 #pragma unroll
-            for (int i = 0; i < BN / 64; ++i)
-              tma_load_2d(st + L.p_bytes + uint32_t(i) * 8192u, &tmQ, fb, n * BN + 64 * i, k0);
+            for (int i = 0; i < BNC / 64; ++i)
+              G::load(st + L.p_bytes + uint32_t(i) * 8192u, &tmQ, fb, qrow0 + 64 * i, k0);
           }
-          if (ttile) {
-            const uint32_t su = st + L.p_bytes + L.q_bytes;
-            if (!MN) {
-              tma_load_2d(su, &tmU, fb, k0, 0);
-            } else {
-              for (int c = 0; c < a.n_rchunks; ++c)
-                tma_load_2d(su + uint32_t(c) * (64u * kRSpan), &tmU, fb, c * RCW, k0);
-            }
-          }
+          if (ttile) G::load(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, int(rank) * u_rows);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         // rank-side operand of the up-projection for this N tile
-        if (!wait_bounded(vempty, (vcount & 1u) ^ 1u, abort_flag, lim, SITE_VEMPTY)) break;
+        if (!wait_bounded(vempty, (vcount & 1u) ^ 1u, abort_flag, lim, SITE_VEMPTY, kClusterScope)) break;
         ++vcount;
         const uint32_t sv = sbase + L.off_v;
-        mbar_arrive_expect_tx(vfull, L.v_bytes);
+        const uint32_t vb = G::leader_addr(vfull);
+        if (leader) mbar_arrive_expect_tx(vfull, L.v_bytes * CG);
         if (!MN) {
           for (int c = 0; c < a.n_rchunks; ++c)
-            tma_load_2d(sv + uint32_t(c) * uint32_t(BN * kRSpan), &tmV, vfull, c * RCW, n * BN);
+            G::load(sv + uint32_t(c) * uint32_t(BNC * kRSpan), &tmV, vb, c * RCW, qrow0);
         } else {
 #pragma unroll
-          for (int i = 0; i < BN / 64; ++i)
-            tma_load_2d(sv + uint32_t(i) * uint32_t(a.r_pad * 128), &tmV, vfull, n * BN + 64 * i, 0);
+          for (int i = 0; i < BNC / 64; ++i)
+            G::load(sv + uint32_t(i) * uint32_t(a.r_pad * 128), &tmV, vb, qrow0 + 64 * i, 0);
         }
       }
       if (*abort_flag) settle_ns(200000);  // let copies in flight land
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
-    if (lane == 0) {
-      const uint32_t id_base = idesc_bf16(kBM, BN, false, MN);
-      const uint32_t id_t = idesc_bf16(kBM, a.r_pad, false, MN);
-      const uint32_t id_up = idesc_bf16(kBM, BN, false, MN);
-      TileSched sch(a);
+    if (lane == 0 && leader) {
+      const uint32_t id_base = idesc_bf16(kBM * CG, BN, false, MN);
+      const uint32_t id_t = idesc_bf16(kBM * CG, a.r_pad, false, false);
+      const uint32_t id_up = idesc_bf16(kBM * CG, BN, false, MN);
+      TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
       uint32_t phase = 0, vcount = 0, ntt = 0, tcount = 0;
       uint32_t acc_waits0 = 0u, acc_waits1 = 0u;  // completed waits per accumulator
@@ -238,44 +326,57 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const bool ttile = (m != prev_m);
         prev_m = m;
         const uint32_t b = tcount & 1u;
-        if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY)) break;
+        if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY, kClusterScope))
+          break;
         uint32_t t_col = 2u * BN;
         if (ttile && borrow) {
           const uint32_t ob = b ^ 1u;
-          if (!wait_bounded(accempty0 + 8u * ob, next_acc_parity(ob), abort_flag, lim, SITE_ACCEMPTY)) break;
+          if (!wait_bounded(accempty0 + 8u * ob, next_acc_parity(ob), abort_flag, lim, SITE_ACCEMPTY,
+                            kClusterScope))
+            break;
           t_col = ob * BN;
         }
         tc_fence_after();
         const uint32_t d_acc = tmem + b * BN;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st = sbase + uint32_t(stage) * L.stage_bytes;
-          const uint32_t sq = st + L.p_bytes;
-          const uint32_t su = sq + L.q_bytes;
+        // The K loop, instantiated twice: with the N = r products of T (first
+        // tile of an M block) and without.  Keeping the plain loop free of
+        // the second MMA stream, and issuing the T products after the base
+        // products of each stage rather than interleaved with them, keeps
+        // the tensor pipe fed (measured: 242 -> 216 us on 8192x4096x4096).
+        auto k_loop = [&](auto with_t) -> bool {
+          constexpr bool kWithT = decltype(with_t)::value;
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL, kClusterScope)) return false;
+            tc_fence_after();
+            const uint32_t st = sbase + uint32_t(stage) * L.stage_bytes;
+            const uint32_t sq = st + L.p_bytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
-            const uint64_t ad = smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
-            const uint64_t bd = MN ? smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B)
-                                   : smem_desc(sq + kk * 32u, 16u, 1024u, SWZ_128B);
-            umma_bf16(d_acc, ad, bd, id_base, acc);
-            if (ttile) {
-              const uint64_t ud = MN ? smem_desc(su + kk * (16u * kRSpan), 64u * kRSpan, 8u * kRSpan, kRSwz)
-                                     : smem_desc(su + kk * 32u, 16u, 1024u, SWZ_128B);
-              umma_bf16(tmem + t_col, ad, ud, id_t, acc);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
+              const uint64_t bd = MN ? smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B)
+                                     : smem_desc(sq + kk * 32u, 16u, 1024u, SWZ_128B);
+              G::mma(d_acc, ad, bd, id_base, (kb | kk) != 0);
             }
+            if constexpr (kWithT) {
+              const uint32_t su = sq + L.q_bytes;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                G::mma(tmem + t_col, smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B),
+                       smem_desc(su + kk * 32u, 16u, 1024u, SWZ_128B), id_t, (kb | kk) != 0);
+            }
+            G::commit_all(empty_bar(stage));
+            if (++stage == S) { stage = 0; phase ^= 1u; }
           }
-          umma_commit(empty_bar(stage));
-          if (++stage == S) { stage = 0; phase ^= 1u; }
-        }
+          return true;
+        };
+        ok = ttile ? k_loop(std::true_type{}) : k_loop(std::false_type{});
         if (!ok) break;
         if (ttile) {
-          umma_commit(tfull);
-          if (!wait_bounded(stfull, ntt & 1u, abort_flag, lim, SITE_STFULL)) break;
+          G::commit_all(tfull);
+          if (!wait_bounded(stfull, ntt & 1u, abort_flag, lim, SITE_STFULL, kClusterScope)) break;
           ++ntt;
         }
-        if (!wait_bounded(vfull, vcount & 1u, abort_flag, lim, SITE_VFULL)) break;
+        if (!wait_bounded(vfull, vcount & 1u, abort_flag, lim, SITE_VFULL, kClusterScope)) break;
         ++vcount;
         tc_fence_after();
         const uint32_t s_t = sbase + L.off_st;
@@ -285,23 +386,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const uint32_t off = uint32_t((kk * 16) % RCW) * 2u;
           const uint64_t ad = smem_desc(s_t + c * uint32_t(kBM * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
           const uint64_t bd = MN ? smem_desc(s_v + uint32_t(kk) * 2048u, uint32_t(a.r_pad) * 128u, 1024u, SWZ_128B)
-                                 : smem_desc(s_v + c * uint32_t(BN * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
-          umma_bf16(d_acc, ad, bd, id_up, 1u);
+                                 : smem_desc(s_v + c * uint32_t(BNC * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
+          G::mma(d_acc, ad, bd, id_up, 1u);
         }
-        umma_commit(vempty);
-        umma_commit(accfull0 + 8u * b);
+        G::commit_all(vempty);
+        G::commit_all(accfull0 + 8u * b);
         ++tcount;
       }
       // make sure no tcgen05 op is still running before TMEM is released
-      umma_commit(drain);
-      wait_bounded(drain, 0u, abort_flag, lim, SITE_DRAIN);
+      G::commit_local(drain);
+      wait_bounded(drain, 0u, abort_flag, lim, SITE_DRAIN, false);
     }
   } else {
     // ---------------------------------------------------- epilogue ----
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int row = q * 32 + lane;     // tile row owned by this thread
     const uint32_t lane_base = uint32_t(q * 32) << 16;
-    TileSched sch(a);
+    TileSched sch(a, n_clusters, cluster_id);
     int m, n, prev_m = -1;
     uint32_t ntt = 0, tcount = 0;
     uint32_t full_waits0 = 0u, full_waits1 = 0u;  // completed accfull waits per buffer
@@ -310,9 +411,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const bool ttile = (m != prev_m);
       prev_m = m;
       const uint32_t b = tcount & 1u;
-      const int grow = m * kBM + row;
+      const int grow = m * (kBM * CG) + int(rank) * kBM + row;
       if (ttile) {
-        if (!warp_wait_bounded(tfull, ntt & 1u, abort_flag, lim, SITE_TFULL)) break;
+        if (!warp_wait_bounded(tfull, ntt & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
         ++ntt;
         tc_fence_after();
         const uint32_t t_col = borrow ? (b ^ 1u) * BN : 2u * BN;
@@ -339,12 +440,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(stfull);
-          if (borrow) mbar_arrive(accempty0 + 8u * (b ^ 1u));
+          G::arrive_leader(stfull);
+          if (borrow) G::arrive_leader(accempty0 + 8u * (b ^ 1u));
         }
       }
       const uint32_t fpar = (b ? full_waits1++ : full_waits0++) & 1u;
-      if (!warp_wait_bounded(accfull0 + 8u * b, fpar, abort_flag, lim, SITE_ACCFULL)) break;
+      if (!warp_wait_bounded(accfull0 + 8u * b, fpar, abort_flag, lim, SITE_ACCFULL, kClusterScope)) break;
       tc_fence_after();
       const uint32_t acc_col = b * BN;
 #pragma unroll 1
@@ -371,17 +472,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty0 + 8u * b);
+      if (lane == 0) G::arrive_leader(accempty0 + 8u * b);
       ++tcount;
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  G::cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    G::dealloc(tmem, 512);
   }
 }
 

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -148,35 +149,82 @@ lora_status_t launch_status() {
 // ------------------------------------------------------------ fused GEMM ----
 
 struct FusedCfg {
-  int BN, RCW, r_pad, n_rchunks, stages, grid;
+  int BN, CG, RCW, r_pad, n_rchunks, stages;
   uint32_t smem;
   FusedArgs args;
 };
+
+// Pipeline stages that fit in shared memory for (BN, CG), capped at 8.
+int fused_stages(int BN, int CG, bool mn, int RCW, int r_pad, int n_rchunks) {
+  const FusedLayout L0(BN, CG, mn, RCW, r_pad, n_rchunks, 0);
+  const uint32_t fixed = L0.total + 1024;
+  if (fixed >= kSmemMax) return 0;
+  return std::min(int((kSmemMax - fixed) / L0.stage_bytes), 8);
+}
+
+// Optional tile override "BN,CG" from LORA_B200_FUSED_TILE (e.g. "256,1"),
+// used to measure or test one configuration; 0,0 = choose per problem.
+void tile_override(int& BN, int& CG) {
+  BN = 0;
+  CG = 0;
+  const char* e = std::getenv("LORA_B200_FUSED_TILE");
+  if (e == nullptr) return;
+  int b = 0, g = 0;
+  if (std::sscanf(e, "%d,%d", &b, &g) == 2 && (b == 128 || b == 256) && (g == 1 || g == 2)) {
+    BN = b;
+    CG = g;
+  }
+}
+
+// Optional schedule override from LORA_B200_FUSED_RUN (-1 = choose).
+int run_override() {
+  const char* e = std::getenv("LORA_B200_FUSED_RUN");
+  if (e == nullptr) return -1;
+  const int v = std::atoi(e);
+  return v >= 0 && v <= 4096 ? v : -1;
+}
 
 bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, FusedCfg& c) {
   c.r_pad = r_pad_of(r);
   c.RCW = rcw_of(c.r_pad);
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
-  const int num_m = int((M + kBM - 1) / kBM);
-  const int cands[2] = {256, 128};
+  int fBN, fCG;
+  tile_override(fBN, fCG);
+  // Preference order: CTA pairs with 256-wide tiles (least operand traffic
+  // per flop), then single CTAs, then 128-wide tiles; take the first that
+  // fits in shared memory and has at least one tile per cluster.
+  const int cands[4][2] = {{256, 2}, {256, 1}, {128, 2}, {128, 1}};
   c.BN = 0;
-  for (int BN : cands) {
-    const FusedLayout L0(BN, mn, c.RCW, c.r_pad, c.n_rchunks, 0);
-    const uint32_t fixed = L0.total + 1024;
-    if (fixed >= kSmemMax) continue;
-    int S = int((kSmemMax - fixed) / L0.stage_bytes);
-    S = std::min(S, 8);
-    const int num_n = int((N + BN - 1) / BN);
-    const bool enough_tiles = (int64_t)num_m * num_n >= sm_count;
-    if (BN == 256 && (S < 3 || !enough_tiles)) continue;
-    if (S < 2) continue;
+  for (int i = 0; i < 4; ++i) {
+    const int BN = cands[i][0], CG = cands[i][1];
+    if (fBN != 0 && (BN != fBN || CG != fCG)) continue;
+    const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks);
+    if (S < (BN == 256 ? 3 : 2)) continue;
+    const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
+    const bool last = (i == 3) || fBN != 0;
+    if (!last && tiles < sm_count / CG) continue;
     c.BN = BN;
+    c.CG = CG;
     c.stages = S;
     break;
   }
+  if (c.BN == 0 && fBN != 0) {
+    // the requested configuration does not fit: choose as usual
+    for (int i = 0; i < 4 && c.BN == 0; ++i) {
+      const int BN = cands[i][0], CG = cands[i][1];
+      const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks);
+      if (S < (BN == 256 ? 3 : 2)) continue;
+      const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
+      if (i < 3 && tiles < sm_count / CG) continue;
+      c.BN = BN;
+      c.CG = CG;
+      c.stages = S;
+    }
+  }
   if (c.BN == 0) return false;
+  const int num_m = int((M + 128 * c.CG - 1) / (128 * c.CG));
   const int num_n = int((N + c.BN - 1) / c.BN);
-  const FusedLayout L(c.BN, mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
+  const FusedLayout L(c.BN, c.CG, mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
   c.smem = L.total + 1024;
   FusedArgs& a = c.args;
   a.M = int32_t(M);
@@ -197,30 +245,89 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
     a.band_w = num_n;
   }
   a.n_bands = (num_n + a.band_w - 1) / a.band_w;
+  const int ro = run_override();
+  a.run_l = ro >= 0 ? ro : 0;
   a.wait_limit_ns = kWaitLimitNs;
-  c.grid = int(std::min<int64_t>(sm_count, (int64_t)num_m * num_n));
   return true;
 }
 
-template <int BN, bool MN, int RCW>
-lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, cudaStream_t st) {
-  auto kern = fused_lora_kernel<BN, MN, RCW>;
+struct ClusterCap {
+  const void* fn;
+  uint32_t smem;
+  int dev;
+  int clusters;
+};
+std::mutex g_cap_mu;
+std::vector<ClusterCap> g_caps;
+
+// How many clusters of `cg` CTAs of this kernel can be resident at once.
+template <typename Kern>
+int max_clusters(Kern kern, int cg, uint32_t smem, int sm_count) {
+  if (cg == 1) return sm_count;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_cap_mu);
+  for (const ClusterCap& cc : g_caps)
+    if (cc.fn == (const void*)kern && cc.smem == smem && cc.dev == dev) return cc.clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(sm_count / cg * cg));
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(cg);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sm_count / cg;
+  }
+  g_caps.push_back(ClusterCap{(const void*)kern, smem, dev, n});
+  return n;
+}
+
+template <int BN, bool MN, int RCW, int CG>
+lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
+  auto kern = fused_lora_kernel<BN, MN, RCW, CG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
     return LORA_ERR_CUDA;
-  kern<<<c.grid, kFusedThreads, c.smem, st>>>(maps[0], maps[1], maps[2], maps[3], c.args);
+  const int64_t tiles = int64_t(c.args.num_m) * c.args.num_n;
+  const int clusters = int(std::min<int64_t>(tiles, max_clusters(kern, CG, c.smem, sm_count)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(clusters * CG));
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(CG);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], c.args) != cudaSuccess)
+    return launch_status();
   return launch_status();
 }
 
-template <bool MN>
-lora_status_t launch_fused(const CUtensorMap* maps, const FusedCfg& c, cudaStream_t st) {
+template <bool MN, int CG>
+lora_status_t launch_fused_cg(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
   if (c.BN == 256) {
-    if (c.RCW == 16) return launch_fused_t<256, MN, 16>(maps, c, st);
-    if (c.RCW == 32) return launch_fused_t<256, MN, 32>(maps, c, st);
-    return launch_fused_t<256, MN, 64>(maps, c, st);
+    if (c.RCW == 16) return launch_fused_t<256, MN, 16, CG>(maps, c, sm_count, st);
+    if (c.RCW == 32) return launch_fused_t<256, MN, 32, CG>(maps, c, sm_count, st);
+    return launch_fused_t<256, MN, 64, CG>(maps, c, sm_count, st);
   }
-  if (c.RCW == 16) return launch_fused_t<128, MN, 16>(maps, c, st);
-  if (c.RCW == 32) return launch_fused_t<128, MN, 32>(maps, c, st);
-  return launch_fused_t<128, MN, 64>(maps, c, st);
+  if (c.RCW == 16) return launch_fused_t<128, MN, 16, CG>(maps, c, sm_count, st);
+  if (c.RCW == 32) return launch_fused_t<128, MN, 32, CG>(maps, c, sm_count, st);
+  return launch_fused_t<128, MN, 64, CG>(maps, c, sm_count, st);
+}
+
+template <bool MN>
+lora_status_t launch_fused(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
+  return c.CG == 2 ? launch_fused_cg<MN, 2>(maps, c, sm_count, st) : launch_fused_cg<MN, 1>(maps, c, sm_count, st);
 }
 
 // ----------------------------------------------------------- skinny GEMM ----
@@ -282,7 +389,7 @@ lora_status_t launch_skinny(const CUtensorMap& p, const CUtensorMap& rm, const S
 
 struct BwdPlan {
   SkinnyCfg t_cfg, db_cfg, da_cfg;
-  size_t off_t, off_dt, off_pb, off_pa, total;
+  size_t off_t, off_dt, off_bt, off_pb, off_pa, total;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -295,7 +402,8 @@ void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
   const size_t tb = align256(size_t(M) * r_pad * 2);
   p.off_t = 0;
   p.off_dt = tb;
-  p.off_pb = 2 * tb;
+  p.off_bt = 2 * tb;                                   // B^T [r, d_out] bf16
+  p.off_pb = p.off_bt + align256(size_t(r) * size_t(d_out) * 2);
   p.off_pa = p.off_pb + align256(size_t(p.db_cfg.splits) * size_t(d_out) * r_pad * 4);
   p.total = p.off_pa + align256(size_t(p.da_cfg.splits) * size_t(d_in) * r_pad * 4);
 }
@@ -477,12 +585,13 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
   c.args.t_out = nullptr;
   CUtensorMap maps[4];
+  const uint32_t bnc = uint32_t(c.BN / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
-      !make_map(&maps[1], W, d_in, d_out, d_in, 64, c.BN, 128) ||
-      !make_map(&maps[2], A, d_in, r, d_in, 64, c.r_pad, 128) ||
-      !make_map(&maps[3], B, r, d_out, r, c.RCW, c.BN, c.RCW * 2))
+      !make_map(&maps[1], W, d_in, d_out, d_in, 64, bnc, 128) ||
+      !make_map(&maps[2], A, d_in, r, d_in, 64, uint32_t(c.r_pad / c.CG), 128) ||
+      !make_map(&maps[3], B, r, d_out, r, c.RCW, bnc, c.RCW * 2))
     return LORA_ERR_CUDA;
-  return launch_fused<false>(maps, c, reinterpret_cast<cudaStream_t>(stream));
+  return launch_fused<false>(maps, c, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r) {
@@ -526,8 +635,13 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
     c.args.scale = 1.0f;
     if ((s = launch_skinny<false, false, false>(mp, mr, c, st)) != LORA_OK) return s;
   }
-  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad])
+  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad]);
+  //    the rank operand of dT is B^T, transposed once into the workspace.
   {
+    __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + p.off_bt);
+    transpose_rank_kernel<<<unsigned((d_out + 31) / 32), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(B), int(d_out), r, Bt);
+    if ((s = launch_status()) != LORA_OK) return s;
     FusedCfg c;
     if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
     c.args.scale = scale;
@@ -536,10 +650,10 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
     CUtensorMap maps[4];
     if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
         !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
-        !make_map(&maps[2], B, r, d_out, r, rcw, 64, rcw * 2) ||
+        !make_map(&maps[2], Bt, d_out, r, d_out, 64, uint32_t(r_pad / c.CG), 128) ||
         !make_map(&maps[3], A, d_in, r, d_in, 64, r_pad, 128))
       return LORA_ERR_CUDA;
-    if ((s = launch_fused<true>(maps, c, st)) != LORA_OK) return s;
+    if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
   }
   // 3. dB partials: sum_m dY[m, i] T[m, j]
   {

@@ -238,3 +238,25 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __res
 }
 
 }  // namespace lora
+
+namespace lora {
+
+// Bt[j, n] = B[n, j] for j < r: the transposed copy of the LoRA B matrix
+// that the dX step reads K-major (B is [d_out, r], Bt is [r, d_out]).
+// Tiles of 32 rows of B through shared memory; r <= 128.
+__global__ void __launch_bounds__(256) transpose_rank_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r,
+                                                              __nv_bfloat16* __restrict__ Bt) {
+  __shared__ __nv_bfloat16 tile[32][129];
+  const int n0 = blockIdx.x * 32;
+  for (int e = threadIdx.x; e < 32 * r; e += blockDim.x) {
+    const int i = e / r, j = e % r;
+    if (n0 + i < d_out) tile[i][j] = B[(size_t)(n0 + i) * r + j];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 32 * r; e += blockDim.x) {
+    const int j = e / 32, i = e % 32;
+    if (n0 + i < d_out) Bt[(size_t)j * d_out + n0 + i] = tile[i][j];
+  }
+}
+
+}  // namespace lora

@@ -91,3 +91,15 @@ def test_bwd_empty_batch_zeroes_adapter_grads(gpu):
     gpu.lora_bwd(X, W, A, B, dY, dX, dA, dB, 32.0, ws)
     assert gpu.lora_get_device_status() == 0
     assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
+
+
+@pytest.mark.parametrize("tile", ["256,2", "256,1", "128,2", "128,1"])
+@pytest.mark.parametrize("run", ["0", "2"])
+@pytest.mark.parametrize("M,d_in,d_out,r,alpha", [(1000, 1544, 1032, 24, 18.0), (777, 2056, 520, 128, 96.0)])
+def test_bwd_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in, d_out, r, alpha):
+    monkeypatch.setenv("LORA_B200_FUSED_TILE", tile)
+    monkeypatch.setenv("LORA_B200_FUSED_RUN", run)
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=13, with_dy=True)
+    dX, dA, dB = run_bwd(gpu, t["X"], t["W"], t["A"], t["B"], t["dY"], alpha)
+    _check_all(t, alpha, dX, dA, dB)

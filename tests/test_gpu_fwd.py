@@ -94,3 +94,22 @@ def test_fwd_empty_batch_is_noop(gpu):
     Y = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     gpu.lora_fwd(X, W, A, B, Y, 32.0)
     assert gpu.lora_get_device_status() == 0
+
+
+TILES = ["256,2", "256,1", "128,2", "128,1"]
+
+
+@pytest.mark.parametrize("tile", TILES)
+@pytest.mark.parametrize("run", ["0", "1", "3"])
+@pytest.mark.parametrize("M,d_in,d_out,r,alpha", [(1000, 1032, 1544, 24, 18.0), (777, 520, 2056, 128, 96.0)])
+def test_fwd_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in, d_out, r, alpha):
+    """Every tile configuration (BN, CTA pair or single CTA) and schedule
+    (contiguous ranges, runs of 1 and 3 N tiles) against the oracle."""
+    monkeypatch.setenv("LORA_B200_FUSED_TILE", tile)
+    monkeypatch.setenv("LORA_B200_FUSED_RUN", run)
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=7)
+    Y = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+    ok, info = lora_tol_check(f64(Y), ref)
+    assert ok, info
