@@ -88,8 +88,8 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
 
 /*
  * Bytes of device scratch lora_bwd needs for this shape (0 when M == 0).
- * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16) and the
- * fp32 split-M partial sums of dA and dB.
+ * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16) and a
+ * transposed copy of B, bf16 [r, d_out].
  */
 size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r);
 
@@ -102,7 +102,8 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
  * `workspace` is caller-owned device memory of at least
  * lora_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on
  * entry do not matter and are clobbered.  Results are bitwise repeatable:
- * the M reduction of dA and dB uses fixed-order partial sums, no atomics.
+ * the M reduction of dA and dB adds fixed per-split partial sums in a fixed
+ * order inside a thread-block cluster, with no atomics.
  * With M == 0, dA and dB are set to zero and nothing else happens.
  */
 lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B,

@@ -308,8 +308,12 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], c.args) != cudaSuccess)
-    return launch_status();
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], c.args);
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "lora_b200: fused launch failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -338,74 +342,90 @@ struct SkinnyCfg {
   SkinnyArgs args;
 };
 
-void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, bool split, SkinnyCfg& c) {
+// Split the contraction so that about two CTAs per SM run; the splits of a
+// row tile form one cluster (at most 8, the portable cluster size), and
+// every split keeps at least 4 K blocks.
+void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, SkinnyCfg& c) {
   c.r_pad = r_pad_of(r);
   c.RCW = rcw_of(c.r_pad);
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
   c.stages = 4;
   const int row_tiles = int((rows + 127) / 128);
   const int nk = int((K + 63) / 64);
-  int splits = 1;
-  if (split) {
-    const int target = 2 * kSplitSMs;
-    splits = std::max(1, std::min((target + row_tiles - 1) / row_tiles, std::max(1, nk / 4)));
-  }
+  const int target = 2 * kSplitSMs;
+  int splits = std::max(1, std::min({(target + row_tiles - 1) / row_tiles, 8, std::max(1, nk / 4)}));
   const int kb_per = std::max(1, (nk + splits - 1) / splits);
   splits = std::max(1, (nk + kb_per - 1) / kb_per);
   c.splits = splits;
   const SkinnyLayout L(r_mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
   c.smem = L.total + 1024;
   SkinnyArgs& a = c.args;
+  std::memset(&a, 0, sizeof(a));
   a.rows = int32_t(rows);
   a.K = int32_t(K);
   a.r_pad = c.r_pad;
+  a.r = r;
   a.n_rchunks = c.n_rchunks;
   a.stages = c.stages;
   a.kb_per_split = kb_per;
+  a.splits = splits;
+  a.out_mode = out_mode;
   a.scale = 1.0f;
-  a.out_bf16 = nullptr;
-  a.out_f32 = nullptr;
   a.wait_limit_ns = kWaitLimitNs;
 }
 
-template <bool P_MN, bool R_MN, bool PARTIALS, int RCW>
+template <bool P_MN, bool R_MN, int RCW>
 lora_status_t launch_skinny_t(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
-  auto kern = skinny_kernel<P_MN, R_MN, RCW, PARTIALS>;
+  auto kern = skinny_kernel<P_MN, R_MN, RCW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
     return LORA_ERR_CUDA;
-  dim3 grid(unsigned((c.args.rows + 127) / 128), unsigned(c.splits));
-  kern<<<grid, 192, c.smem, st>>>(p, rm, c.args);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((c.args.rows + 127) / 128), unsigned(c.splits));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = unsigned(c.splits);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, rm, c.args);
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "lora_b200: skinny launch failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
   return launch_status();
 }
 
-template <bool P_MN, bool R_MN, bool PARTIALS>
+template <bool P_MN, bool R_MN>
 lora_status_t launch_skinny(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
-  if (c.RCW == 16) return launch_skinny_t<P_MN, R_MN, PARTIALS, 16>(p, rm, c, st);
-  if (c.RCW == 32) return launch_skinny_t<P_MN, R_MN, PARTIALS, 32>(p, rm, c, st);
-  return launch_skinny_t<P_MN, R_MN, PARTIALS, 64>(p, rm, c, st);
+  if (c.RCW == 16) return launch_skinny_t<P_MN, R_MN, 16>(p, rm, c, st);
+  if (c.RCW == 32) return launch_skinny_t<P_MN, R_MN, 32>(p, rm, c, st);
+  return launch_skinny_t<P_MN, R_MN, 64>(p, rm, c, st);
 }
 
 // --------------------------------------------------------- bwd workspace ----
 
 struct BwdPlan {
   SkinnyCfg t_cfg, db_cfg, da_cfg;
-  size_t off_t, off_dt, off_bt, off_pb, off_pa, total;
+  size_t off_t, off_dt, off_bt, total;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
-  pick_skinny(M, d_in, r, false, false, p.t_cfg);
-  pick_skinny(d_out, M, r, true, true, p.db_cfg);
-  pick_skinny(d_in, M, r, true, true, p.da_cfg);
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, p.t_cfg);
+  pick_skinny(d_out, M, r, true, OUT_ROWS_R, p.db_cfg);
+  pick_skinny(d_in, M, r, true, OUT_COLS_R, p.da_cfg);
   const int r_pad = r_pad_of(r);
   const size_t tb = align256(size_t(M) * r_pad * 2);
-  p.off_t = 0;
-  p.off_dt = tb;
-  p.off_bt = 2 * tb;                                   // B^T [r, d_out] bf16
-  p.off_pb = p.off_bt + align256(size_t(r) * size_t(d_out) * 2);
-  p.off_pa = p.off_pb + align256(size_t(p.db_cfg.splits) * size_t(d_out) * r_pad * 4);
-  p.total = p.off_pa + align256(size_t(p.da_cfg.splits) * size_t(d_in) * r_pad * 4);
+  p.off_t = 0;                                         // T   bf16 [M, r_pad]
+  p.off_dt = tb;                                       // dT  bf16 [M, r_pad]
+  p.off_bt = 2 * tb;                                   // B^T bf16 [r, d_out]
+  p.total = p.off_bt + align256(size_t(r) * size_t(d_out) * 2);
 }
 
 // -------------------------------------------------------- merge batching ----
@@ -619,29 +639,27 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_t);
   __nv_bfloat16* dTws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_dt);
-  float* partB = reinterpret_cast<float*>(ws + p.off_pb);
-  float* partA = reinterpret_cast<float*>(ws + p.off_pa);
+  __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + p.off_bt);
   const float scale = alpha / float(r);
   const int r_pad = r_pad_of(r);
   const int rcw = rcw_of(r_pad);
 
-  // 1. T = X A^T (recomputed), bf16 [M, r_pad]
+  // 1. T = X A^T (recomputed), bf16 [M, r_pad]; the same launch writes
+  //    B^T [r, d_out], the K-major rank operand of the dX step.
   {
     CUtensorMap mp, mr;
     if (!make_map(&mp, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr, A, d_in, r, d_in, 64, r_pad, 128))
       return LORA_ERR_CUDA;
     SkinnyCfg c = p.t_cfg;
-    c.args.out_bf16 = Tws;
-    c.args.scale = 1.0f;
-    if ((s = launch_skinny<false, false, false>(mp, mr, c, st)) != LORA_OK) return s;
+    c.args.out = Tws;
+    c.args.tr_src = reinterpret_cast<const __nv_bfloat16*>(B);
+    c.args.tr_dst = Bt;
+    c.args.tr_rows = int32_t(d_out);
+    c.args.tr_r = r;
+    if ((s = launch_skinny<false, false>(mp, mr, c, st)) != LORA_OK) return s;
   }
-  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad]);
-  //    the rank operand of dT is B^T, transposed once into the workspace.
+  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad])
   {
-    __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + p.off_bt);
-    transpose_rank_kernel<<<unsigned((d_out + 31) / 32), 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(B), int(d_out), r, Bt);
-    if ((s = launch_status()) != LORA_OK) return s;
     FusedCfg c;
     if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
     c.args.scale = scale;
@@ -655,31 +673,26 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
       return LORA_ERR_CUDA;
     if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
   }
-  // 3. dB partials: sum_m dY[m, i] T[m, j]
+  // 3. dB = s * sum_m dY[m, i] T[m, j]
   {
     CUtensorMap mp, mr;
     if (!make_map(&mp, dY, d_out, M, d_out, 64, 64, 128) || !make_map(&mr, Tws, r_pad, M, r_pad, rcw, 64, rcw * 2))
       return LORA_ERR_CUDA;
     SkinnyCfg c = p.db_cfg;
-    c.args.out_f32 = partB;
-    if ((s = launch_skinny<true, true, true>(mp, mr, c, st)) != LORA_OK) return s;
+    c.args.out = reinterpret_cast<__nv_bfloat16*>(dB);
+    c.args.scale = scale;
+    if ((s = launch_skinny<true, true>(mp, mr, c, st)) != LORA_OK) return s;
   }
-  // 4. dA^T partials: sum_m X[m, i] dT[m, j]
+  // 4. dA^T[i, j] = sum_m X[m, i] dT[m, j], written transposed into dA
   {
     CUtensorMap mp, mr;
     if (!make_map(&mp, X, d_in, M, d_in, 64, 64, 128) || !make_map(&mr, dTws, r_pad, M, r_pad, rcw, 64, rcw * 2))
       return LORA_ERR_CUDA;
     SkinnyCfg c = p.da_cfg;
-    c.args.out_f32 = partA;
-    if ((s = launch_skinny<true, true, true>(mp, mr, c, st)) != LORA_OK) return s;
+    c.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
+    if ((s = launch_skinny<true, true>(mp, mr, c, st)) != LORA_OK) return s;
   }
-  // 5. fixed-order reductions: dB = s * sum, dA = (sum)^T
-  reduce_partials_kernel<<<unsigned((d_out + 31) / 32), 256, 0, st>>>(
-      partB, p.db_cfg.splits, int(d_out), r_pad, r, scale, reinterpret_cast<__nv_bfloat16*>(dB), 0);
-  if ((s = launch_status()) != LORA_OK) return s;
-  reduce_partials_kernel<<<unsigned((d_in + 31) / 32), 256, 0, st>>>(
-      partA, p.da_cfg.splits, int(d_in), r_pad, r, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), 1);
-  return launch_status();
+  return LORA_OK;
 }
 
 lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,

@@ -322,3 +322,17 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 }
 
 }  // namespace lora
+
+namespace lora {
+
+// 16-byte load from another CTA's shared memory (shared::cluster address).
+__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+}  // namespace lora

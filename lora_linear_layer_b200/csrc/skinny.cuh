@@ -1,40 +1,63 @@
 // skinny.cuh - OUT[i, j] = scale * sum_k P(i, k) R(j, k) with j < r_pad.
 //
 // The rank-sized products of the backward (fastaf 0.1.0, "BWD kernel
-// speedup": the dA and dB kernels; the M reduction made sequence-parallel):
+// speedup": the dA and dB kernels, with the M reduction made parallel):
 //   T recompute:  P = X[M, d_in] (K-major),  R = A[r, d_in] (K-major)
-//   dB partials:  P(i,k) = dY[k, i] (MN),    R(j,k) = T[k, j] (MN)
-//   dA partials:  P(i,k) = X[k, i] (MN),     R(j,k) = dT[k, j] (MN)
-// i runs over 128-row tiles (UMMA M = 128), the rank is the UMMA N, and the
-// contraction K (tokens for dA/dB) is split across blockIdx.y into
-// fixed ranges.  Each split writes its fp32 partial; reduce_partials sums
-// them in split order, so the result does not depend on scheduling.
+//   dB:           P(i,k) = dY[k, i] (MN),    R(j,k) = T[k, j] (MN)
+//   dA:           P(i,k) = X[k, i] (MN),     R(j,k) = dT[k, j] (MN)
+// i runs over 128-row tiles (UMMA M = 128) and the rank is the UMMA N.  The
+// contraction K (d_in for T, tokens for dA/dB) is split into S fixed ranges
+// (blockIdx.y).  The S CTAs of one row tile form a cluster: each leaves its
+// fp32 partial in its own shared memory, then each reduces 1/S of the rows,
+// reading the S partials over distributed shared memory and adding them in
+// split order, before one rounding to bf16.
+// Nothing goes through global memory and no atomics are used, so results
+// are bitwise repeatable for a given shape.
 #pragma once
 
 #include "common.cuh"
 
 namespace lora {
 
+enum SkinnyOut : int32_t {
+  OUT_ROWS_RPAD = 0,   // out[i * r_pad + j], every j < r_pad       (T)
+  OUT_ROWS_R = 1,      // out[i * r + j], j < r                     (dB)
+  OUT_COLS_R = 2,      // out[j * rows + i], j < r (transposed)     (dA)
+};
+
 struct SkinnyArgs {
   int32_t rows;           // number of output rows (size of the i dimension)
   int32_t K;              // contraction length
   int32_t r_pad;          // rank rounded up to 16
+  int32_t r;              // rank
   int32_t n_rchunks;      // r_pad / RCW rounded up
   int32_t stages;
   int32_t kb_per_split;   // K blocks (of 64) per split
-  float scale;            // applied in the bf16 mode
-  __nv_bfloat16* out_bf16;  // mode bf16: [rows, r_pad]
-  float* out_f32;           // mode partials: [splits, rows, r_pad]
+  int32_t splits;         // gridDim.y; the cluster size when > 1
+  int32_t out_mode;       // SkinnyOut
+  float scale;            // applied to the reduced fp32 sum before rounding
+  __nv_bfloat16* out;
+  // optional side job of the split-0 CTAs: Bt[j, n] = B[n, j] for n < tr_rows,
+  // j < tr_r (the transposed copy of B that the dX step reads)
+  const __nv_bfloat16* tr_src;
+  __nv_bfloat16* tr_dst;
+  int32_t tr_rows, tr_r;
   uint64_t wait_limit_ns;
 };
 
 struct SkinnyLayout {
-  uint32_t p_bytes, r_bytes, stage_bytes, off_bar, total;
+  uint32_t p_bytes, r_bytes, stage_bytes, ring_bytes, red_stride, red_bytes, off_bar, total;
   __host__ __device__ SkinnyLayout(bool r_mn, int rcw, int r_pad, int n_rchunks, int stages) {
     p_bytes = 128 * 64 * 2;
     r_bytes = r_mn ? uint32_t(n_rchunks * rcw * 128) : uint32_t(r_pad * 128);
     stage_bytes = p_bytes + r_bytes;
-    off_bar = stage_bytes * stages;
+    ring_bytes = stage_bytes * stages;
+    // fp32 partial rows, padded by 4 floats so the 16-byte accesses of 8
+    // consecutive rows fall in distinct bank groups
+    red_stride = uint32_t((r_pad + 4) * 4);
+    red_bytes = 128u * red_stride;
+    const uint32_t body = ring_bytes > red_bytes ? ring_bytes : red_bytes;  // the partial reuses the ring
+    off_bar = (body + 1023u) & ~1023u;
     total = off_bar + 256;
   }
 };
@@ -45,7 +68,7 @@ __host__ __device__ inline uint32_t tmem_cols_for(int r_pad) {
   return c;
 }
 
-template <bool P_MN, bool R_MN, int RCW, bool PARTIALS>
+template <bool P_MN, bool R_MN, int RCW>
 __global__ void __launch_bounds__(192, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmR,
                   const SkinnyArgs a) {
@@ -69,6 +92,7 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t ncols = tmem_cols_for(a.r_pad);
+  const bool clustered = a.splits > 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -90,8 +114,9 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   const int i0 = blockIdx.x * 128;
+  const int split = blockIdx.y;
   const int nk_total = (a.K + 63) / 64;
-  const int kb0 = blockIdx.y * a.kb_per_split;
+  const int kb0 = split * a.kb_per_split;
   const int kb1 = imin(nk_total, kb0 + a.kb_per_split);
   const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
   const uint64_t lim = a.wait_limit_ns;
@@ -149,17 +174,47 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(drain);
       wait_bounded(drain, 0u, abort_flag, lim, SITE_DRAIN);
     }
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int gi = i0 + row;
-    const uint32_t lane_base = uint32_t(q * 32) << 16;
+  }
+
+  // ---------------------------------------------- partial / output -----
+  const int q = warp & 3;
+  const int row = q * 32 + lane;
+  const int gi = i0 + row;
+  auto write_out = [&](const float* acc, int col0) {  // 16 reduced values of row gi
+    if (gi >= a.rows) return;
+    if (a.out_mode == OUT_ROWS_RPAD) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(acc[2 * e] * a.scale, acc[2 * e + 1] * a.scale);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)gi * a.r_pad + col0);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    } else if (a.out_mode == OUT_ROWS_R) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {               // 8 values = 16 bytes, r % 8 == 0
+        if (col0 + 8 * h >= a.r) break;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          pk[e] = pack_bf16x2(acc[8 * h + 2 * e] * a.scale, acc[8 * h + 2 * e + 1] * a.scale);
+        *reinterpret_cast<uint4*>(a.out + (size_t)gi * a.r + col0 + 8 * h) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (col0 + e < a.r) a.out[(size_t)(col0 + e) * a.rows + gi] = __float2bfloat16_rn(acc[e] * a.scale);
+    }
+  };
+
+  uint8_t* const red = gbase;  // fp32 partial rows (reuses the ring once the MMAs are done)
+  if (warp >= 2) {
     bool have = true;
     if (nkb > 0) {
       have = warp_wait_bounded(accfull, 0u, abort_flag, lim, SITE_ACCFULL);
       tc_fence_after();
     }
     if (have) {
+      const uint32_t lane_base = uint32_t(q * 32) << 16;
       for (int col = 0; col < a.r_pad; col += 16) {
         uint32_t v[16];
         if (nkb > 0) {
@@ -167,95 +222,87 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = 0u;  // empty split: contributes zero
+          for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty split: contributes zero
         }
-        if (gi < a.rows) {
-          if (PARTIALS) {
-            float* dst = a.out_f32 + ((size_t)blockIdx.y * a.rows + gi) * a.r_pad + col;
+        if (!clustered) {
+          float acc[16];
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-              reinterpret_cast<uint4*>(dst)[g] = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-          } else {
-            uint32_t pk[8];
+          for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(v[e]);
+          write_out(acc, col);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(red + row * L.red_stride + col * 4);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * a.scale, __uint_as_float(v[2 * i + 1]) * a.scale);
-            uint4* dst = reinterpret_cast<uint4*>(a.out_bf16 + (size_t)gi * a.r_pad + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
+          for (int g = 0; g < 4; ++g) dst[g] = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
         }
+      }
+    }
+    // side job: transposed copy of B, one slice per row tile (split 0 only)
+    if (a.tr_src != nullptr && split == 0) {
+      const int per = (a.tr_rows + int(gridDim.x) - 1) / int(gridDim.x);
+      const int n0 = int(blockIdx.x) * per;
+      const int n1 = imin(a.tr_rows, n0 + per);
+      for (int e = int(threadIdx.x) - 64; e < (n1 - n0) * a.tr_r; e += 128) {
+        const int n = n0 + e / a.tr_r, j = e % a.tr_r;
+        a.tr_dst[(size_t)j * a.tr_rows + n] = a.tr_src[(size_t)n * a.tr_r + j];
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (clustered) {
+    cluster_barrier_sync();  // every split's partial is in its shared memory
+    // Every CTA of the cluster reduces its own slice of the 128 rows: one
+    // float4 (4 consecutive columns) per task, the S partials loaded
+    // together and added in split order.
+    if (warp >= 2 && !*abort_flag) {
+      const int S = a.splits;
+      const int f4_per_row = a.r_pad / 4;
+      const int rows_per = (128 + S - 1) / S;
+      const int r0 = split * rows_per;
+      const int r1 = imin(128, r0 + rows_per);
+      for (int task = int(threadIdx.x) - 64; task < (r1 - r0) * f4_per_row; task += 128) {
+        const int rr = r0 + task / f4_per_row;
+        const int c4 = task % f4_per_row;
+        const uint32_t off = smem_addr(red + rr * L.red_stride + c4 * 16);
+        float4 p[8];
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S) p[s2] = ld_shared_cluster_f4(mapa_shared(off, uint32_t(s2)));
+        float4 acc = p[0];
+#pragma unroll
+        for (int s2 = 1; s2 < 8; ++s2)
+          if (s2 < S) {
+            acc.x += p[s2].x;
+            acc.y += p[s2].y;
+            acc.z += p[s2].z;
+            acc.w += p[s2].w;
+          }
+        const int g = i0 + rr;
+        const int j0 = c4 * 4;
+        if (g < a.rows) {
+          const float v[4] = {acc.x * a.scale, acc.y * a.scale, acc.z * a.scale, acc.w * a.scale};
+          if (a.out_mode == OUT_ROWS_RPAD) {
+            *reinterpret_cast<uint2*>(a.out + (size_t)g * a.r_pad + j0) =
+                make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+          } else if (a.out_mode == OUT_ROWS_R) {
+            if (j0 < a.r)  // r % 8 == 0, so the 4 columns are all in or all out
+              *reinterpret_cast<uint2*>(a.out + (size_t)g * a.r + j0) =
+                  make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (j0 + e < a.r) a.out[(size_t)(j0 + e) * a.rows + g] = __float2bfloat16_rn(v[e]);
+          }
+        }
+      }
+    }
+    cluster_barrier_sync();  // peers keep their shared memory until every slice is done
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
-  }
-}
-
-// dst = bf16(scale * sum_{s < splits} part[s]) in split order.
-//   part: [splits, rows, r_pad] fp32.  Only j < r is written.
-//   transpose = false: dst[i * r + j]       (dB: [d_out, r])
-//   transpose = true:  dst[j * rows + i]    (dA: [r, d_in])
-// One block covers 32 rows x r_pad; the transposed case goes through shared
-// memory so both the reads and the writes are coalesced.
-__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ part, int splits,
-                                                               int rows, int r_pad, int r, float scale,
-                                                               __nv_bfloat16* __restrict__ dst, int transpose) {
-  __shared__ float tile[32][257];
-  const int i0 = blockIdx.x * 32;
-  const int nelem = 32 * r_pad;
-  const size_t plane = (size_t)rows * r_pad;
-  for (int e = threadIdx.x; e < nelem; e += blockDim.x) {
-    const int i = i0 + e / r_pad;
-    const int j = e % r_pad;
-    float acc = 0.f;
-    if (i < rows) {
-      const float* p = part + (size_t)i * r_pad + j;
-      for (int s = 0; s < splits; ++s) acc += p[(size_t)s * plane];
-    }
-    acc *= scale;
-    if (!transpose) {
-      if (i < rows && j < r) dst[(size_t)i * r + j] = __float2bfloat16_rn(acc);
-    } else {
-      tile[e / r_pad][j] = acc;
-    }
-  }
-  if (transpose) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < nelem; e += blockDim.x) {
-      const int j = e / 32;
-      const int ii = e % 32;
-      const int i = i0 + ii;
-      if (j < r && i < rows) dst[(size_t)j * rows + i] = __float2bfloat16_rn(tile[ii][j]);
-    }
-  }
-}
-
-}  // namespace lora
-
-namespace lora {
-
-// Bt[j, n] = B[n, j] for j < r: the transposed copy of the LoRA B matrix
-// that the dX step reads K-major (B is [d_out, r], Bt is [r, d_out]).
-// Tiles of 32 rows of B through shared memory; r <= 128.
-__global__ void __launch_bounds__(256) transpose_rank_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r,
-                                                              __nv_bfloat16* __restrict__ Bt) {
-  __shared__ __nv_bfloat16 tile[32][129];
-  const int n0 = blockIdx.x * 32;
-  for (int e = threadIdx.x; e < 32 * r; e += blockDim.x) {
-    const int i = e / r, j = e % r;
-    if (n0 + i < d_out) tile[i][j] = B[(size_t)(n0 + i) * r + j];
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 32 * r; e += blockDim.x) {
-    const int j = e / 32, i = e % 32;
-    if (n0 + i < d_out) Bt[(size_t)j * d_out + n0 + i] = tile[i][j];
   }
 }
 
