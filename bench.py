@@ -240,6 +240,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     import lora_linear_layer_b200 as L
+    from lora_linear_layer_b200 import dp
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -273,8 +274,7 @@ def run_ours(args):
             ev_f1.record(stream)
         L.lora_bwd(X, W, A, B, dY, dX, dA, dB, alpha, ws, stream)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            dp.allreduce_adapter_grads(dA, dB)   # the data-parallel exchange (NCCL)
         L.lora_merge(W, A, B, Wm, alpha, stream)
 
     warm = max(3, args.warmup)
@@ -310,10 +310,7 @@ def run_ours(args):
     fwd_ms = [f0.elapsed_time(f1) for (_, _, f0, f1) in ev]
     total_ms = sum(step_ms)
     fwd_avg_ms = sum(fwd_ms) / K
-    t_local = torch.tensor([total_ms, fwd_avg_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    total_ms, fwd_avg_ms = float(t_local[0]), float(t_local[1])
+    total_ms, fwd_avg_ms = dp.max_over_ranks([total_ms, fwd_avg_ms], device="cuda")
 
     # ---------------- end to end through the C ABI with host buffers -------
     e2e = None
@@ -346,10 +343,8 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": step_flops(sh) * Ke * world / (float(e_ms[0]) * 1e-3) / 1e12, "unit": UNIT,
+        e_ms = dp.max_over_ranks([e0.elapsed_time(e1)], device="cuda")[0]
+        e2e = {"value": step_flops(sh) * Ke * world / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": Ke,
                "what": "every step copies X, W, A, B, dY from pinned host memory and reads dA, dB back"}
 
@@ -394,6 +389,82 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------- extra modes ----
+
+def _time_events(fn, flush, n, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    return ts[len(ts) // 2], ts[max(0, len(ts) // 10)], ts[min(len(ts) - 1, (9 * len(ts)) // 10)]
+
+
+def run_sweep(args):
+    """lora_fwd on every point of the square sweep: one JSON line per point
+    with us/call (median, p10, p90), TFLOP/s, GB/s of the minimum bytes and
+    the fraction of the binding roof (tensor or HBM, measured peaks)."""
+    import torch
+    import lora_linear_layer_b200 as L
+    peaks, src = load_peaks()
+    P = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12
+    BW = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for idx, sh in enumerate(WL.sweep_points()):
+        if args.sweep_filter and args.sweep_filter not in sh.name:
+            continue
+        t = WL.make_layer_inputs(sh, seed=idx)
+        X, W, A, B = (t[k].cuda() for k in ("X", "W", "A", "B"))
+        Y = torch.empty((sh.M, sh.d_out), dtype=torch.bfloat16, device="cuda")
+        med, p10, p90 = _time_events(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, args.steps)
+        F = flops_fwd(sh.M, sh.d_in, sh.d_out, sh.r)
+        by = 2.0 * (sh.M * sh.d_in + sh.d_out * sh.d_in + sh.r * (sh.d_in + sh.d_out) + sh.M * sh.d_out)
+        t_roof = max(F / P, by / BW)
+        print(json.dumps({"point": sh.name, "M": sh.M, "d": sh.d_in, "r": sh.r, "us_median": med, "us_p10": p10,
+                          "us_p90": p90, "tflops": F / med / 1e6, "gbs_min_bytes": by / med / 1e3,
+                          "bound": "tensor" if F / P >= by / BW else "hbm", "roof_frac": t_roof * 1e6 / med,
+                          "peaks": f"bf16 burst and HBM copy ({src})"}), flush=True)
+        del X, W, A, B, Y
+    return 0
+
+
+def run_merge(args):
+    """The 36-layer x 7-target adapter merge (r = 32): one batched
+    restore-and-merge refresh from the pristine copies per cycle."""
+    import torch
+    import lora_linear_layer_b200 as L
+    peaks, src = load_peaks()
+    BW = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+    r, alpha = WL.MERGE_R, WL.MERGE_ALPHA
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(0)
+    items, nbytes = [], 0.0
+    for s in WL.merge_shapes():
+        d_out, d_in = s["d_out"], s["d_in"]
+        W = (torch.randn(d_out, d_in, generator=gen, device="cuda") * d_in ** -0.5).to(torch.bfloat16)
+        A = (torch.randn(r, d_in, generator=gen, device="cuda") * d_in ** -0.5).to(torch.bfloat16)
+        B = (torch.randn(d_out, r, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        items.append((W, A, B, torch.empty_like(W)))
+        nbytes += 4.0 * d_out * d_in + 2.0 * r * (d_in + d_out)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    med, p10, p90 = _time_events(lambda: L.lora_merge_batched(items, r, alpha), flush, args.steps)
+    print(json.dumps({"workload": "merge 36 layers x 7 targets, hidden 2560, r=32", "matrices": len(items),
+                      "ms_per_cycle": med / 1e3, "ms_p10": p10 / 1e3, "ms_p90": p90 / 1e3,
+                      "gbs": nbytes / med / 1e3, "hbm_frac": nbytes / med / 1e3 / (BW / 1e9),
+                      "bytes_per_cycle": nbytes, "peak": f"HBM copy {BW/1e9:.0f} GB/s ({src})",
+                      "inputs": "seeded torch.randn on the device (timing only; parity in tests)"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -404,7 +475,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--sweep", action="store_true", help="time lora_fwd on every sweep point (one line each)")
+    ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
+    ap.add_argument("--merge", action="store_true", help="time the 252-matrix batched merge refresh")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
+    if args.merge:
+        return run_merge(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -119,9 +119,34 @@ CUtensorMapSwizzle swz_enum(uint32_t span_bytes) {
 }
 
 // 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
-// row pitch `ld` elements, box {box_inner, box_outer}.
+// row pitch `ld` elements, box {box_inner, box_outer}.  Encoded maps are
+// kept in a small per-thread cache keyed by every encoding input, so a
+// layer called again on the same buffers skips the driver call.
+struct MapKey {
+  const void* ptr;
+  uint64_t inner, outer, ld;
+  uint32_t bi, bo, swz;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && inner == o.inner && outer == o.outer && ld == o.ld && bi == o.bi && bo == o.bo &&
+           swz == o.swz;
+  }
+};
+constexpr int kMapCache = 64;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  int used = 0, next = 0;
+};
+thread_local MapCache t_maps;
+
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
               uint32_t box_outer, uint32_t swz_span_bytes) {
+  const MapKey k{ptr, inner, outer, ld, box_inner, box_outer, swz_span_bytes};
+  for (int i = 0; i < t_maps.used; ++i)
+    if (t_maps.key[i] == k) {
+      *m = t_maps.map[i];
+      return true;
+    }
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -134,6 +159,32 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
                  (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
     return false;
   }
+  const int slot = t_maps.used < kMapCache ? t_maps.used++ : (t_maps.next++ % kMapCache);
+  t_maps.key[slot] = k;
+  t_maps.map[slot] = *m;
+  return true;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel, device
+// and size (the attribute only grows).
+std::mutex g_attr_mu;
+std::vector<std::pair<std::pair<const void*, int>, int>> g_attr_done;
+
+template <typename Kern>
+bool ensure_smem_attr(Kern kern, uint32_t smem) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  for (auto& e : g_attr_done)
+    if (e.first.first == fn && e.first.second == dev && e.second >= int(smem)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) return false;
+  for (auto& e : g_attr_done)
+    if (e.first.first == fn && e.first.second == dev) {
+      e.second = int(smem);
+      return true;
+    }
+  g_attr_done.push_back({{fn, dev}, int(smem)});
   return true;
 }
 
@@ -292,8 +343,7 @@ int max_clusters(Kern kern, int cg, uint32_t smem, int sm_count) {
 template <int BN, bool MN, int RCW, int CG>
 lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
   auto kern = fused_lora_kernel<BN, MN, RCW, CG>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
-    return LORA_ERR_CUDA;
+  if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
   const int64_t tiles = int64_t(c.args.num_m) * c.args.num_n;
   const int clusters = int(std::min<int64_t>(tiles, max_clusters(kern, CG, c.smem, sm_count)));
   cudaLaunchConfig_t cfg = {};
@@ -377,8 +427,7 @@ void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, Skinny
 template <bool P_MN, bool R_MN, int RCW>
 lora_status_t launch_skinny_t(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
   auto kern = skinny_kernel<P_MN, R_MN, RCW>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) != cudaSuccess)
-    return LORA_ERR_CUDA;
+  if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned((c.args.rows + 127) / 128), unsigned(c.splits));
   cfg.blockDim = dim3(192);
@@ -455,8 +504,7 @@ lora_status_t check_merge_item(const MergeItem& it, int32_t r) {
 template <int RCW>
 lora_status_t launch_merge_t(const MergeTable& tab, int total_tiles, uint32_t smem, cudaStream_t st) {
   auto kern = merge_kernel<RCW>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return LORA_ERR_CUDA;
+  if (!ensure_smem_attr(kern, smem)) return LORA_ERR_CUDA;
   kern<<<total_tiles, 192, smem, st>>>(tab);
   return launch_status();
 }
