@@ -21,7 +21,8 @@
 //     write it into shared memory in the UMMA K-major swizzled layout (it
 //     never goes to global memory in the forward);
 //   * one more MMA pass (K = r) accumulates (sT) V^T onto the base
-//     accumulator; the epilogue rounds once to bf16 and stores.
+//     accumulator; the epilogue rounds once to bf16 and writes OUT with
+//     TMA stores of 32 x 32 boxes staged in shared memory.
 // T is kept in shared memory and reused for every further tile of the same
 // M block the CTA processes.  Warp roles: warp 0 = TMA producer, warp 1 =
 // MMA issuer and TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes
@@ -45,6 +46,8 @@ namespace lora {
 constexpr int kBM = 128;          // rows per CTA (UMMA M per CTA)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr int kFusedThreads = 192;
+constexpr int kEpCols = 32;                    // output columns per epilogue store
+constexpr uint32_t kEpBufBytes = 32u * kEpCols * 2u;  // one warp's 32 rows, 64-byte swizzle
 
 struct FusedArgs {
   int32_t M, N, K;          // OUT is [M, N]; contraction length K
@@ -62,8 +65,8 @@ struct FusedArgs {
 
 // Byte sizes / offsets of one CTA's shared-memory carve-up (host and device).
 struct FusedLayout {
-  uint32_t p_bytes, q_bytes, u_bytes, stage_bytes, v_bytes, st_bytes;
-  uint32_t off_v, off_st, off_bar, total;
+  uint32_t p_bytes, q_bytes, u_bytes, stage_bytes, v_bytes, st_bytes, ep_bytes;
+  uint32_t off_v, off_st, off_ep, off_bar, total;
   __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages) {
     const int bnc = BN / CG;            // Q / V rows held by this CTA
     p_bytes = kBM * kBK * 2;
@@ -73,8 +76,10 @@ struct FusedLayout {
     v_bytes = mn ? uint32_t((bnc / 64) * r_pad * 128) : uint32_t(n_rchunks * bnc * rcw * 2);
     st_bytes = uint32_t(n_rchunks * kBM * rcw * 2);
     off_v = stage_bytes * stages;
+    ep_bytes = 4u * kEpBufBytes;
     off_st = off_v + v_bytes;
-    off_bar = off_st + st_bytes;
+    off_ep = off_st + st_bytes;
+    off_bar = off_ep + ep_bytes;
     total = off_bar + 256;
   }
 };
@@ -180,7 +185,7 @@ template <int BN, bool MN, int RCW, int CG>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_lora_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
-                      const FusedArgs a) {
+                      const __grid_constant__ CUtensorMap tmO, const FusedArgs a) {
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(CG == 1 || CG == 2, "CG");
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
@@ -240,6 +245,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     tma_prefetch_desc(&tmU);
     tma_prefetch_desc(&tmV);
   }
+  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmO);
   if (warp == 1) G::alloc(smem_addr(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
@@ -407,6 +413,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint32_t ntt = 0, tcount = 0;
     uint32_t full_waits0 = 0u, full_waits1 = 0u;  // completed accfull waits per buffer
     uint8_t* const st_ptr = gbase + L.off_st;
+    uint8_t* const ep_ptr = gbase + L.off_ep + q * kEpBufBytes;
+    const uint32_t ep_buf = sbase + L.off_ep + uint32_t(q) * kEpBufBytes;
     while (sch.next(m, n)) {
       const bool ttile = (m != prev_m);
       prev_m = m;
@@ -448,26 +456,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       if (!warp_wait_bounded(accfull0 + 8u * b, fpar, abort_flag, lim, SITE_ACCFULL, kClusterScope)) break;
       tc_fence_after();
       const uint32_t acc_col = b * BN;
+      // Each 32-column chunk: TMEM -> registers -> bf16 -> this warp's
+      // swizzled staging buffer -> one TMA store of 32 rows x 64 bytes
+      // (rows past M and columns past N are clipped by the tensor map).
+      const int wrow0 = m * (kBM * CG) + int(rank) * kBM + q * 32;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = 0; ch < BN / kEpCols; ++ch) {
         uint32_t v[32];
-        tmem_ld_x32(tmem + lane_base + acc_col + uint32_t(ch * 32), v);
+        tmem_ld_x32(tmem + lane_base + acc_col + uint32_t(ch * kEpCols), v);
         tmem_ld_wait();
-        if (grow < a.M) {
-          const int col0 = n * BN + ch * 32;
-          __nv_bfloat16* orow = a.out + (size_t)grow * a.N;
+        const int col0 = n * BN + ch * kEpCols;
+        if (col0 >= a.N || wrow0 >= a.M) continue;
+        uint4 pk[4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + 8 * g;
-            if (col < a.N) {
-              uint4 pk;
-              pk.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
-              pk.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
-              pk.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
-              pk.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
-              *reinterpret_cast<uint4*>(orow + col) = pk;
-            }
-          }
+        for (int g = 0; g < 4; ++g) {
+          pk[g].x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
+          pk[g].y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
+          pk[g].z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
+          pk[g].w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
+        }
+        if (lane == 0) bulk_wait_group_read0();  // the previous store has read the buffer
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          *reinterpret_cast<uint4*>(ep_ptr + swz_offset(uint32_t(lane), uint32_t(g), kEpCols * 2)) = pk[g];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmO, ep_buf, col0, wrow0);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
@@ -475,6 +492,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       if (lane == 0) G::arrive_leader(accempty0 + 8u * b);
       ++tcount;
     }
+    if (lane == 0) bulk_wait_group0();  // every output store has completed
   }
 
   tc_fence_before();

@@ -292,6 +292,10 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   if (footprint > 96.0e6) {
     const double per_ntile = double(c.BN) * double(K) * 2.0;
     a.band_w = std::max(1, std::min(num_n, int(40.0e6 / per_ntile)));
+    // a band must still hold two tiles per cluster: with few M blocks the
+    // operands are not reused across the band anyway
+    const int want = int((2 * (sm_count / c.CG) + num_m - 1) / num_m);
+    a.band_w = std::max(a.band_w, std::min(num_n, want));
   } else {
     a.band_w = num_n;
   }
@@ -358,7 +362,7 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], c.args);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], c.args);
   if (e != cudaSuccess) {
     std::fprintf(stderr, "lora_b200: fused launch failed: %s\n", cudaGetErrorString(e));
     cudaGetLastError();
@@ -652,12 +656,13 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
   c.args.scale = alpha / float(r);
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
   c.args.t_out = nullptr;
-  CUtensorMap maps[4];
+  CUtensorMap maps[5];
   const uint32_t bnc = uint32_t(c.BN / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
       !make_map(&maps[1], W, d_in, d_out, d_in, 64, bnc, 128) ||
       !make_map(&maps[2], A, d_in, r, d_in, 64, uint32_t(c.r_pad / c.CG), 128) ||
-      !make_map(&maps[3], B, r, d_out, r, c.RCW, bnc, c.RCW * 2))
+      !make_map(&maps[3], B, r, d_out, r, c.RCW, bnc, c.RCW * 2) ||
+      !make_map(&maps[4], Y, d_out, M, d_out, kEpCols, 32, kEpCols * 2))
     return LORA_ERR_CUDA;
   return launch_fused<false>(maps, c, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -713,11 +718,12 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
     c.args.scale = scale;
     c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
     c.args.t_out = dTws;
-    CUtensorMap maps[4];
+    CUtensorMap maps[5];
     if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
         !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
         !make_map(&maps[2], Bt, d_out, r, d_out, 64, uint32_t(r_pad / c.CG), 128) ||
-        !make_map(&maps[3], A, d_in, r, d_in, 64, r_pad, 128))
+        !make_map(&maps[3], A, d_in, r, d_in, 64, r_pad, 128) ||
+        !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
       return LORA_ERR_CUDA;
     if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
   }
