@@ -4,9 +4,11 @@
 One step = one pass of the whole hot path over one batch of synthetic
 input: lora_fwd (Y), lora_bwd (dX, dA, dB; T recomputed) and lora_merge
 (W' = W + s B A) on the attention-projection workload X[8192, 4096],
-W[4096, 4096], r = 16, alpha = 32.  With N > 1 GPUs every rank runs the
-same step on its own batch (data parallel along M, weak scaling) and the
-adapter gradients dA, dB are summed across ranks with one NCCL all-reduce.
+W[4096, 4096], r = 16, alpha = 32 (or, with --workload mlp_up, the MLP
+up-projection X[16384, 4096], W[14336, 4096], r = 64, alpha = 128).
+With N > 1 GPUs every rank runs the same step on its own batch (data
+parallel along M, weak scaling) and the adapter gradients dA, dB are summed
+across ranks with one NCCL all-reduce.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -34,7 +36,8 @@ import workloads as WL  # noqa: E402
 
 METRIC = "fused LoRA fwd/bwd TFLOP/s (bf16) and % of B200 dense peak; µs/call"
 UNIT = "TFLOP/s"
-WORKLOAD = WL.ATTN_PROJ
+# the step's workload: attention projection by default, --workload mlp_up for the MLP up-projection
+WORKLOADS = {"attn_proj": WL.ATTN_PROJ, "mlp_up": WL.MLP_UP}
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
@@ -206,7 +209,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sh = WORKLOAD
+    sh = WORKLOADS[args.workload]
     rows = 512
     t = WL.make_layer_inputs(WL.LayerShape(rows, sh.d_in, sh.d_out, sh.r, sh.alpha), seed=0, with_dy=True)
     for _ in range(max(args.warmup, 0)):
@@ -253,7 +256,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     L.lib()
 
-    sh = WORKLOAD
+    sh = WORKLOADS[args.workload]
     M, d_in, d_out, r, alpha = sh.M, sh.d_in, sh.d_out, sh.r, sh.alpha
     host = WL.make_layer_inputs(sh, seed=rank, with_dy=True)
     X, W, A, B, dY = (host[k].cuda() for k in ("X", "W", "A", "B", "dY"))
@@ -471,6 +474,9 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=tuple(WORKLOADS), default="attn_proj",
+                    help="attn_proj: X[8192,4096] W[4096,4096] r=16 (default); "
+                         "mlp_up: X[16384,4096] W[14336,4096] r=64")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

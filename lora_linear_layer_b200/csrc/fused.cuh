@@ -54,6 +54,7 @@ struct FusedArgs {
   int32_t r_pad;            // rank rounded up to 16 (UMMA N of the T product)
   int32_t n_rchunks;        // r_pad / RCW rounded up
   int32_t stages;           // pipeline depth
+  int32_t ep_bufs;          // output staging buffers per epilogue warp (1 or 2)
   float scale;              // s = alpha / r
   __nv_bfloat16* out;       // [M, N] row-major, ld = N
   __nv_bfloat16* t_out;     // optional [M, r_pad] bf16 copy of s*T (dT), or null
@@ -67,7 +68,8 @@ struct FusedArgs {
 struct FusedLayout {
   uint32_t p_bytes, q_bytes, u_bytes, stage_bytes, v_bytes, st_bytes, ep_bytes;
   uint32_t off_v, off_st, off_ep, off_bar, total;
-  __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages) {
+  __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages,
+                                  int ep_bufs) {
     const int bnc = BN / CG;            // Q / V rows held by this CTA
     p_bytes = kBM * kBK * 2;
     q_bytes = uint32_t(bnc * kBK * 2);
@@ -76,7 +78,7 @@ struct FusedLayout {
     v_bytes = mn ? uint32_t((bnc / 64) * r_pad * 128) : uint32_t(n_rchunks * bnc * rcw * 2);
     st_bytes = uint32_t(n_rchunks * kBM * rcw * 2);
     off_v = stage_bytes * stages;
-    ep_bytes = 4u * kEpBufBytes;
+    ep_bytes = 4u * uint32_t(ep_bufs) * kEpBufBytes;
     off_st = off_v + v_bytes;
     off_ep = off_st + st_bytes;
     off_bar = off_ep + ep_bytes;
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (sbase - raw);
 
-  const FusedLayout L(BN, CG, MN, RCW, a.r_pad, a.n_rchunks, a.stages);
+  const FusedLayout L(BN, CG, MN, RCW, a.r_pad, a.n_rchunks, a.stages, a.ep_bufs);
   const int S = a.stages;
   const uint32_t bar0 = sbase + L.off_bar;
   // barrier map (8 bytes each); full / vfull / accempty / stfull / drain
@@ -413,8 +415,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint32_t ntt = 0, tcount = 0;
     uint32_t full_waits0 = 0u, full_waits1 = 0u;  // completed accfull waits per buffer
     uint8_t* const st_ptr = gbase + L.off_st;
-    uint8_t* const ep_ptr = gbase + L.off_ep + q * kEpBufBytes;
-    const uint32_t ep_buf = sbase + L.off_ep + uint32_t(q) * kEpBufBytes;
+    // this warp's output staging buffers (used in turn when there are two)
+    const uint32_t ep_off = L.off_ep + uint32_t(q * a.ep_bufs) * kEpBufBytes;
+    uint32_t epc = 0;  // output blocks staged so far
     while (sch.next(m, n)) {
       const bool ttile = (m != prev_m);
       prev_m = m;
@@ -475,15 +478,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           pk[g].z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
           pk[g].w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
         }
-        if (lane == 0) bulk_wait_group_read0();  // the previous store has read the buffer
+        // the store that last used this buffer has read it
+        if (lane == 0) {
+          if (a.ep_bufs == 2) bulk_wait_group_read1();
+          else bulk_wait_group_read0();
+        }
         __syncwarp();
+        const uint32_t bo = ep_off + (a.ep_bufs == 2 ? (epc & 1u) * kEpBufBytes : 0u);
+        ++epc;
 #pragma unroll
         for (int g = 0; g < 4; ++g)
-          *reinterpret_cast<uint4*>(ep_ptr + swz_offset(uint32_t(lane), uint32_t(g), kEpCols * 2)) = pk[g];
+          *reinterpret_cast<uint4*>(gbase + bo + swz_offset(uint32_t(lane), uint32_t(g), kEpCols * 2)) = pk[g];
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmO, ep_buf, col0, wrow0);
+          tma_store_2d(&tmO, sbase + bo, col0, wrow0);
           bulk_commit_group();
         }
       }

@@ -200,14 +200,14 @@ lora_status_t launch_status() {
 // ------------------------------------------------------------ fused GEMM ----
 
 struct FusedCfg {
-  int BN, CG, RCW, r_pad, n_rchunks, stages;
+  int BN, CG, RCW, r_pad, n_rchunks, stages, ep_bufs;
   uint32_t smem;
   FusedArgs args;
 };
 
 // Pipeline stages that fit in shared memory for (BN, CG), capped at 8.
-int fused_stages(int BN, int CG, bool mn, int RCW, int r_pad, int n_rchunks) {
-  const FusedLayout L0(BN, CG, mn, RCW, r_pad, n_rchunks, 0);
+int fused_stages(int BN, int CG, bool mn, int RCW, int r_pad, int n_rchunks, int ep_bufs) {
+  const FusedLayout L0(BN, CG, mn, RCW, r_pad, n_rchunks, 0, ep_bufs);
   const uint32_t fixed = L0.total + 1024;
   if (fixed >= kSmemMax) return 0;
   return std::min(int((kSmemMax - fixed) / L0.stage_bytes), 8);
@@ -249,7 +249,7 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   for (int i = 0; i < 4; ++i) {
     const int BN = cands[i][0], CG = cands[i][1];
     if (fBN != 0 && (BN != fBN || CG != fCG)) continue;
-    const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks);
+    const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks, 1);
     if (S < (BN == 256 ? 3 : 2)) continue;
     const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
     const bool last = (i == 3) || fBN != 0;
@@ -263,7 +263,7 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
     // the requested configuration does not fit: choose as usual
     for (int i = 0; i < 4 && c.BN == 0; ++i) {
       const int BN = cands[i][0], CG = cands[i][1];
-      const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks);
+      const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks, 1);
       if (S < (BN == 256 ? 3 : 2)) continue;
       const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
       if (i < 3 && tiles < sm_count / CG) continue;
@@ -275,7 +275,9 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   if (c.BN == 0) return false;
   const int num_m = int((M + 128 * c.CG - 1) / (128 * c.CG));
   const int num_n = int((N + c.BN - 1) / c.BN);
-  const FusedLayout L(c.BN, c.CG, mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
+  // a second output staging buffer per epilogue warp when it costs no stage
+  c.ep_bufs = fused_stages(c.BN, c.CG, mn, c.RCW, c.r_pad, c.n_rchunks, 2) >= c.stages ? 2 : 1;
+  const FusedLayout L(c.BN, c.CG, mn, c.RCW, c.r_pad, c.n_rchunks, c.stages, c.ep_bufs);
   c.smem = L.total + 1024;
   FusedArgs& a = c.args;
   a.M = int32_t(M);
@@ -284,6 +286,7 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   a.r_pad = c.r_pad;
   a.n_rchunks = c.n_rchunks;
   a.stages = c.stages;
+  a.ep_bufs = c.ep_bufs;
   a.num_m = num_m;
   a.num_n = num_n;
   // Column bands keep the operands the whole GPU touches at once well
