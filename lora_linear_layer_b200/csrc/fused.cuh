@@ -254,6 +254,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   G::cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above touches no global memory, so it may overlap the
+  // previous kernel on the stream; every global access comes after the wait.
+  griddep_launch_dependents();
+  griddep_wait();
 
   // T accumulator placement: its own columns if two BN-wide accumulators
   // and r_pad columns fit in 512, else it borrows the other accumulator.

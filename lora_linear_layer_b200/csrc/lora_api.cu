@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/lora.h"
@@ -197,6 +198,53 @@ lora_status_t launch_status() {
   return LORA_OK;
 }
 
+// Programmatic dependent launch (PDL) on every launch unless
+// LORA_B200_PDL=0: a kernel's prologue (barrier init, TMEM allocation,
+// descriptor prefetch) then overlaps the tail of the kernel before it on the
+// stream.  Every kernel waits (griddepcontrol.wait) before its first global
+// memory access, so results do not depend on this setting.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("LORA_B200_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+// cudaLaunchKernelEx with an optional cluster shape and the PDL attribute.
+template <typename... KArgs, typename... Args>
+lora_status_t launch_ex(const char* what, void (*kern)(KArgs...), dim3 grid, dim3 block, uint32_t smem,
+                        cudaStream_t st, const dim3* cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster != nullptr) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster->x;
+    attr[n].val.clusterDim.y = cluster->y;
+    attr[n].val.clusterDim.z = cluster->z;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "lora_b200: %s launch failed: %s\n", what, cudaGetErrorString(e));
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // ------------------------------------------------------------ fused GEMM ----
 
 struct FusedCfg {
@@ -353,25 +401,9 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
   if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
   const int64_t tiles = int64_t(c.args.num_m) * c.args.num_n;
   const int clusters = int(std::min<int64_t>(tiles, max_clusters(kern, CG, c.smem, sm_count)));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(clusters * CG));
-  cfg.blockDim = dim3(kFusedThreads);
-  cfg.dynamicSmemBytes = c.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(CG);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], c.args);
-  if (e != cudaSuccess) {
-    std::fprintf(stderr, "lora_b200: fused launch failed: %s\n", cudaGetErrorString(e));
-    cudaGetLastError();
-    return LORA_ERR_CUDA;
-  }
-  return launch_status();
+  const dim3 cl(unsigned(CG), 1, 1);
+  return launch_ex("fused", kern, dim3(unsigned(clusters * CG)), dim3(kFusedThreads), c.smem, st, &cl, maps[0],
+                   maps[1], maps[2], maps[3], maps[4], c.args);
 }
 
 template <bool MN, int CG>
@@ -435,25 +467,9 @@ template <bool P_MN, bool R_MN, int RCW>
 lora_status_t launch_skinny_t(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
   auto kern = skinny_kernel<P_MN, R_MN, RCW>;
   if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned((c.args.rows + 127) / 128), unsigned(c.splits));
-  cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = c.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = unsigned(c.splits);
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, rm, c.args);
-  if (e != cudaSuccess) {
-    std::fprintf(stderr, "lora_b200: skinny launch failed: %s\n", cudaGetErrorString(e));
-    cudaGetLastError();
-    return LORA_ERR_CUDA;
-  }
-  return launch_status();
+  const dim3 cl(1, unsigned(c.splits), 1);
+  return launch_ex("skinny", kern, dim3(unsigned((c.args.rows + 127) / 128), unsigned(c.splits)), dim3(192), c.smem,
+                   st, &cl, p, rm, c.args);
 }
 
 template <bool P_MN, bool R_MN>
@@ -512,8 +528,7 @@ template <int RCW>
 lora_status_t launch_merge_t(const MergeTable& tab, int total_tiles, uint32_t smem, cudaStream_t st) {
   auto kern = merge_kernel<RCW>;
   if (!ensure_smem_attr(kern, smem)) return LORA_ERR_CUDA;
-  kern<<<total_tiles, 192, smem, st>>>(tab);
-  return launch_status();
+  return launch_ex("merge", kern, dim3(unsigned(total_tiles)), dim3(192), smem, st, nullptr, tab);
 }
 
 lora_status_t run_merge(const MergeItem* items, int n, int32_t r, float alpha, cudaStream_t st) {
@@ -559,8 +574,8 @@ lora_status_t zero_bytes(void* p, size_t bytes, cudaStream_t st) {
   if ((bytes % 16) != 0 || !aligned16(p)) return LORA_ERR_ALIGN;
   const size_t n16 = bytes / 16;
   const int blocks = int(std::min<size_t>((n16 + 255) / 256, 4096));
-  zero16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<uint4*>(p), n16);
-  return launch_status();
+  return launch_ex("zero", zero16_kernel, dim3(unsigned(blocks)), dim3(256), 0, st, nullptr,
+                   reinterpret_cast<uint4*>(p), n16);
 }
 
 }  // namespace
@@ -793,15 +808,16 @@ lora_status_t lora_restore(const void* W_src, void* W_dst, int64_t n_elems, void
   const size_t n16 = size_t(n_elems) * 2 / 16;
   if (n16 > 0) {
     const int blocks = int(std::min<size_t>((n16 + 255) / 256, size_t(dev.sm_count) * 8));
-    copy16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(W_src), reinterpret_cast<uint4*>(W_dst), n16);
-    if ((s = launch_status()) != LORA_OK) return s;
+    s = launch_ex("copy", copy16_kernel, dim3(unsigned(blocks)), dim3(256), 0, st, nullptr,
+                  reinterpret_cast<const uint4*>(W_src), reinterpret_cast<uint4*>(W_dst), n16);
+    if (s != LORA_OK) return s;
   }
   const size_t done = n16 * 8;
   const size_t rest = size_t(n_elems) - done;
   if (rest > 0) {
-    copy2_kernel<<<1, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(W_src) + done,
-                                    reinterpret_cast<uint16_t*>(W_dst) + done, rest);
-    if ((s = launch_status()) != LORA_OK) return s;
+    s = launch_ex("copy", copy2_kernel, dim3(1), dim3(256), 0, st, nullptr,
+                  reinterpret_cast<const uint16_t*>(W_src) + done, reinterpret_cast<uint16_t*>(W_dst) + done, rest);
+    if (s != LORA_OK) return s;
   }
   return LORA_OK;
 }

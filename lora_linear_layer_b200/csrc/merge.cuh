@@ -99,6 +99,10 @@ __global__ void __launch_bounds__(192) merge_kernel(const __grid_constant__ Merg
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above touches no global memory, so it may overlap the
+  // previous kernel on the stream; every global access comes after the wait.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -182,17 +186,23 @@ __global__ void __launch_bounds__(192) merge_kernel(const __grid_constant__ Merg
 
 // W_dst <- W_src, 16 bytes per thread per step (restore from pristine).
 __global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+  griddep_launch_dependents();
+  griddep_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
     dst[i] = src[i];
 }
 
 // Tail of a copy that is not a multiple of 16 bytes (2-byte elements).
 __global__ void copy2_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
+  griddep_launch_dependents();
+  griddep_wait();
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = src[i];
 }
 
 __global__ void zero16_kernel(uint4* __restrict__ dst, size_t n16) {
+  griddep_launch_dependents();
+  griddep_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
     dst[i] = make_uint4(0u, 0u, 0u, 0u);
 }

@@ -94,6 +94,19 @@ __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel on
+// the stream be scheduled once every CTA of this grid has executed it (or
+// exited); wait blocks until the previous kernel on the stream has completed
+// and its memory operations are visible.  Both are no-ops for a kernel
+// launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (TMA stores, tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

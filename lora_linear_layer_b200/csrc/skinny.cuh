@@ -112,6 +112,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The prologue above touches no global memory, so it may overlap the
+  // previous kernel on the stream; every global access comes after the wait.
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int i0 = blockIdx.x * 128;
   const int split = blockIdx.y;
