@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
                   "lora_linear_layer_b200/csrc/common.cuh")
-LAUNCHES_PER_STEP = 6   # fwd 1; bwd: T (+ B transpose), dX, dB, dA; merge 1
+LAUNCHES_PER_STEP = 5   # fwd 1; bwd: T (+ B transpose), dX, dB + dA; merge 1
 
 
 # ------------------------------------------------------ algorithmic work ----

@@ -45,6 +45,7 @@ using namespace lora;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitimate wait
 constexpr uint32_t kSmemMax = 232448;             // 227 KB opt-in dynamic shared memory
 constexpr int kSplitSMs = 148;                    // B200 SM count used to size split-M work
+constexpr uint32_t kSmemPerSM = 233472;           // shared memory per SM (228 KB)
 
 // ------------------------------------------------------------ validation ----
 
@@ -434,20 +435,26 @@ struct SkinnyCfg {
 // Split the contraction so that about two CTAs per SM run; the splits of a
 // row tile form one cluster (at most 8, the portable cluster size), and
 // every split keeps at least 4 K blocks.
-void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, SkinnyCfg& c) {
+// `launch_tiles` is the number of 128-row tiles of the whole launch (both
+// jobs when dB and dA share one), which sets the split count: as many
+// splits as keep every resident CTA slot of the GPU busy, at most 8 (the
+// portable cluster size) and at least 4 K blocks per split.
+void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, int64_t launch_tiles, SkinnyCfg& c) {
   c.r_pad = r_pad_of(r);
   c.RCW = rcw_of(c.r_pad);
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
   c.stages = 4;
-  const int row_tiles = int((rows + 127) / 128);
+  const SkinnyLayout L(r_mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
+  c.smem = L.total + 1024;
+  const int per_sm = std::max(1, std::min<int>(int(kSmemPerSM / (c.smem + 1024)),
+                                               int(512 / tmem_cols_for(c.r_pad))));
+  const int slots = per_sm * kSplitSMs;
+  const int tiles = int(std::max<int64_t>(1, launch_tiles));
   const int nk = int((K + 63) / 64);
-  const int target = 2 * kSplitSMs;
-  int splits = std::max(1, std::min({(target + row_tiles - 1) / row_tiles, 8, std::max(1, nk / 4)}));
+  int splits = std::max(1, std::min({slots / tiles, 8, std::max(1, nk / 4)}));
   const int kb_per = std::max(1, (nk + splits - 1) / splits);
   splits = std::max(1, (nk + kb_per - 1) / kb_per);
   c.splits = splits;
-  const SkinnyLayout L(r_mn, c.RCW, c.r_pad, c.n_rchunks, c.stages);
-  c.smem = L.total + 1024;
   SkinnyArgs& a = c.args;
   std::memset(&a, 0, sizeof(a));
   a.rows = int32_t(rows);
@@ -463,20 +470,28 @@ void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, Skinny
   a.wait_limit_ns = kWaitLimitNs;
 }
 
+// One launch of one job (c1 == nullptr) or of two jobs with the same
+// template arguments, split count and shared-memory layout.
 template <bool P_MN, bool R_MN, int RCW>
-lora_status_t launch_skinny_t(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
+lora_status_t launch_skinny_t(const CUtensorMap& p0, const CUtensorMap& r0, const SkinnyCfg& c0,
+                              const CUtensorMap* p1, const CUtensorMap* r1, const SkinnyCfg* c1, cudaStream_t st) {
   auto kern = skinny_kernel<P_MN, R_MN, RCW>;
-  if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
-  const dim3 cl(1, unsigned(c.splits), 1);
-  return launch_ex("skinny", kern, dim3(unsigned((c.args.rows + 127) / 128), unsigned(c.splits)), dim3(192), c.smem,
-                   st, &cl, p, rm, c.args);
+  if (!ensure_smem_attr(kern, c0.smem)) return LORA_ERR_CUDA;
+  const int t0 = (c0.args.rows + 127) / 128;
+  const int t1 = c1 != nullptr ? (c1->args.rows + 127) / 128 : 0;
+  const dim3 cl(1, unsigned(c0.splits), 1);
+  return launch_ex("skinny", kern, dim3(unsigned(t0 + t1), unsigned(c0.splits)), dim3(192), c0.smem, st, &cl, p0, r0,
+                   p1 != nullptr ? *p1 : p0, r1 != nullptr ? *r1 : r0, c0.args, c1 != nullptr ? c1->args : c0.args,
+                   int32_t(t0));
 }
 
 template <bool P_MN, bool R_MN>
-lora_status_t launch_skinny(const CUtensorMap& p, const CUtensorMap& rm, const SkinnyCfg& c, cudaStream_t st) {
-  if (c.RCW == 16) return launch_skinny_t<P_MN, R_MN, 16>(p, rm, c, st);
-  if (c.RCW == 32) return launch_skinny_t<P_MN, R_MN, 32>(p, rm, c, st);
-  return launch_skinny_t<P_MN, R_MN, 64>(p, rm, c, st);
+lora_status_t launch_skinny(const CUtensorMap& p0, const CUtensorMap& r0, const SkinnyCfg& c0, cudaStream_t st,
+                            const CUtensorMap* p1 = nullptr, const CUtensorMap* r1 = nullptr,
+                            const SkinnyCfg* c1 = nullptr) {
+  if (c0.RCW == 16) return launch_skinny_t<P_MN, R_MN, 16>(p0, r0, c0, p1, r1, c1, st);
+  if (c0.RCW == 32) return launch_skinny_t<P_MN, R_MN, 32>(p0, r0, c0, p1, r1, c1, st);
+  return launch_skinny_t<P_MN, R_MN, 64>(p0, r0, c0, p1, r1, c1, st);
 }
 
 // --------------------------------------------------------- bwd workspace ----
@@ -489,9 +504,11 @@ struct BwdPlan {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
-  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, p.t_cfg);
-  pick_skinny(d_out, M, r, true, OUT_ROWS_R, p.db_cfg);
-  pick_skinny(d_in, M, r, true, OUT_COLS_R, p.da_cfg);
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, (M + 127) / 128, p.t_cfg);
+  // dB and dA share one launch, so they share its split count
+  const int64_t dbda_tiles = (d_out + 127) / 128 + (d_in + 127) / 128;
+  pick_skinny(d_out, M, r, true, OUT_ROWS_R, dbda_tiles, p.db_cfg);
+  pick_skinny(d_in, M, r, true, OUT_COLS_R, dbda_tiles, p.da_cfg);
   const int r_pad = r_pad_of(r);
   const size_t tb = align256(size_t(M) * r_pad * 2);
   p.off_t = 0;                                         // T   bf16 [M, r_pad]
@@ -745,24 +762,21 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
       return LORA_ERR_CUDA;
     if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
   }
-  // 3. dB = s * sum_m dY[m, i] T[m, j]
+  // 3 + 4, one launch:  dB = s * sum_m dY[m, i] T[m, j]  and
+  //                     dA^T[i, j] = sum_m X[m, i] dT[m, j], written transposed into dA
   {
-    CUtensorMap mp, mr;
-    if (!make_map(&mp, dY, d_out, M, d_out, 64, 64, 128) || !make_map(&mr, Tws, r_pad, M, r_pad, rcw, 64, rcw * 2))
+    CUtensorMap mp_b, mr_b, mp_a, mr_a;
+    if (!make_map(&mp_b, dY, d_out, M, d_out, 64, 64, 128) ||
+        !make_map(&mr_b, Tws, r_pad, M, r_pad, rcw, 64, rcw * 2) ||
+        !make_map(&mp_a, X, d_in, M, d_in, 64, 64, 128) ||
+        !make_map(&mr_a, dTws, r_pad, M, r_pad, rcw, 64, rcw * 2))
       return LORA_ERR_CUDA;
-    SkinnyCfg c = p.db_cfg;
-    c.args.out = reinterpret_cast<__nv_bfloat16*>(dB);
-    c.args.scale = scale;
-    if ((s = launch_skinny<true, true>(mp, mr, c, st)) != LORA_OK) return s;
-  }
-  // 4. dA^T[i, j] = sum_m X[m, i] dT[m, j], written transposed into dA
-  {
-    CUtensorMap mp, mr;
-    if (!make_map(&mp, X, d_in, M, d_in, 64, 64, 128) || !make_map(&mr, dTws, r_pad, M, r_pad, rcw, 64, rcw * 2))
-      return LORA_ERR_CUDA;
-    SkinnyCfg c = p.da_cfg;
-    c.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
-    if ((s = launch_skinny<true, true>(mp, mr, c, st)) != LORA_OK) return s;
+    SkinnyCfg cb = p.db_cfg;
+    cb.args.out = reinterpret_cast<__nv_bfloat16*>(dB);
+    cb.args.scale = scale;
+    SkinnyCfg ca = p.da_cfg;
+    ca.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
+    if ((s = launch_skinny<true, true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
   }
   return LORA_OK;
 }

@@ -13,6 +13,8 @@
 // split order, before one rounding to bf16.
 // Nothing goes through global memory and no atomics are used, so results
 // are bitwise repeatable for a given shape.
+// One launch can carry two independent jobs of the same form (dB and dA):
+// row tiles [0, x_split) of the grid run job 0, the rest job 1.
 #pragma once
 
 #include "common.cuh"
@@ -70,8 +72,15 @@ __host__ __device__ inline uint32_t tmem_cols_for(int r_pad) {
 
 template <bool P_MN, bool R_MN, int RCW>
 __global__ void __launch_bounds__(192, 1)
-    skinny_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmR,
-                  const SkinnyArgs a) {
+    skinny_kernel(const __grid_constant__ CUtensorMap tmP0, const __grid_constant__ CUtensorMap tmR0,
+                  const __grid_constant__ CUtensorMap tmP1, const __grid_constant__ CUtensorMap tmR1,
+                  const __grid_constant__ SkinnyArgs a0, const __grid_constant__ SkinnyArgs a1, const int32_t x_split) {
+  const bool second = int(blockIdx.x) >= x_split;
+  const SkinnyArgs& a = second ? a1 : a0;
+  const CUtensorMap* const tmP = second ? &tmP1 : &tmP0;
+  const CUtensorMap* const tmR = second ? &tmR1 : &tmR0;
+  const int bx = second ? int(blockIdx.x) - x_split : int(blockIdx.x);   // row tile within the job
+  const int job_tiles = second ? int(gridDim.x) - x_split : x_split;
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
   constexpr uint32_t kRSpan = RCW * 2;
 
@@ -117,7 +126,7 @@ __global__ void __launch_bounds__(192, 1)
   griddep_launch_dependents();
   griddep_wait();
 
-  const int i0 = blockIdx.x * 128;
+  const int i0 = bx * 128;
   const int split = blockIdx.y;
   const int nk_total = (a.K + 63) / 64;
   const int kb0 = split * a.kb_per_split;
@@ -136,17 +145,17 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(fb, L.stage_bytes);
         const int k0 = kb * 64;
         if (!P_MN) {
-          tma_load_2d(st, &tmP, fb, k0, i0);
+          tma_load_2d(st, tmP, fb, k0, i0);
         } else {
-          tma_load_2d(st, &tmP, fb, i0, k0);
-          tma_load_2d(st + 8192u, &tmP, fb, i0 + 64, k0);
+          tma_load_2d(st, tmP, fb, i0, k0);
+          tma_load_2d(st + 8192u, tmP, fb, i0 + 64, k0);
         }
         const uint32_t sr = st + L.p_bytes;
         if (!R_MN) {
-          tma_load_2d(sr, &tmR, fb, k0, 0);
+          tma_load_2d(sr, tmR, fb, k0, 0);
         } else {
           for (int c = 0; c < a.n_rchunks; ++c)
-            tma_load_2d(sr + uint32_t(c) * (64u * kRSpan), &tmR, fb, c * RCW, k0);
+            tma_load_2d(sr + uint32_t(c) * (64u * kRSpan), tmR, fb, c * RCW, k0);
         }
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
@@ -212,6 +221,17 @@ __global__ void __launch_bounds__(192, 1)
 
   uint8_t* const red = gbase;  // fp32 partial rows (reuses the ring once the MMAs are done)
   if (warp >= 2) {
+    // side job while the K loop runs: transposed copy of B, one slice per
+    // row tile (split 0 only)
+    if (a.tr_src != nullptr && split == 0) {
+      const int per = (a.tr_rows + job_tiles - 1) / job_tiles;
+      const int n0 = bx * per;
+      const int n1 = imin(a.tr_rows, n0 + per);
+      for (int e = int(threadIdx.x) - 64; e < (n1 - n0) * a.tr_r; e += 128) {
+        const int n = n0 + e / a.tr_r, j = e % a.tr_r;
+        a.tr_dst[(size_t)j * a.tr_rows + n] = a.tr_src[(size_t)n * a.tr_r + j];
+      }
+    }
     bool have = true;
     if (nkb > 0) {
       have = warp_wait_bounded(accfull, 0u, abort_flag, lim, SITE_ACCFULL);
@@ -238,16 +258,6 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int g = 0; g < 4; ++g) dst[g] = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
         }
-      }
-    }
-    // side job: transposed copy of B, one slice per row tile (split 0 only)
-    if (a.tr_src != nullptr && split == 0) {
-      const int per = (a.tr_rows + int(gridDim.x) - 1) / int(gridDim.x);
-      const int n0 = int(blockIdx.x) * per;
-      const int n1 = imin(a.tr_rows, n0 + per);
-      for (int e = int(threadIdx.x) - 64; e < (n1 - n0) * a.tr_r; e += 128) {
-        const int n = n0 + e / a.tr_r, j = e % a.tr_r;
-        a.tr_dst[(size_t)j * a.tr_rows + n] = a.tr_src[(size_t)n * a.tr_r + j];
       }
     }
   }
