@@ -20,6 +20,7 @@
 #include "fused.cuh"
 #include "merge.cuh"
 #include "skinny.cuh"
+#include "splitk.cuh"
 
 namespace lora {
 
@@ -424,6 +425,81 @@ lora_status_t launch_fused(const CUtensorMap* maps, const FusedCfg& c, int sm_co
   return c.CG == 2 ? launch_fused_cg<MN, 2>(maps, c, sm_count, st) : launch_fused_cg<MN, 1>(maps, c, sm_count, st);
 }
 
+// ------------------------------------------------- split-K fused forward ----
+
+struct SplitkCfg {
+  int RCW;
+  uint32_t smem;
+  SplitkArgs args;
+};
+
+// LORA_B200_SPLITK=0 turns the split-K forward off, =1 uses it whenever it
+// applies at all (S >= 2); unset: automatic.  A forced fused tile
+// (LORA_B200_FUSED_TILE) also turns it off.
+int splitk_mode() {
+  const char* e = std::getenv("LORA_B200_SPLITK");
+  if (e != nullptr && (e[0] == '0' || e[0] == '1')) return e[0] - '0';
+  return std::getenv("LORA_B200_FUSED_TILE") != nullptr ? 0 : -1;
+}
+
+// The split-K forward is used when 128 x 128 tiles would fill at most half of
+// the SMs: S CTAs (2..8, the portable cluster size) share each tile, with at
+// least 8 K blocks each (shorter K loops do not pay for the reduction:
+// measured slower at K = 512 and at 4 K blocks per split), and a rank of at
+// most 64 (at r = 128 the T reduction costs more than the split saves).
+bool pick_splitk(int64_t M, int64_t N, int64_t K, int r, int sm_count, SplitkCfg& c) {
+  const int mode = splitk_mode();
+  if (mode == 0) return false;
+  const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
+  if (tiles > 65535) return false;
+  if (mode < 0 && (tiles * 2 > sm_count || r_pad_of(r) > 64)) return false;
+  const int nk = int((K + 63) / 64);
+  int S = int(std::min<int64_t>({8, std::max<int64_t>(1, sm_count / tiles), nk / 8}));
+  if (S < 2) return false;
+  const int kb_per = (nk + S - 1) / S;
+  S = (nk + kb_per - 1) / kb_per;
+  if (S < 2) return false;
+  const int r_pad = r_pad_of(r);
+  c.RCW = rcw_of(r_pad);
+  const int n_rchunks = (r_pad + c.RCW - 1) / c.RCW;
+  const SplitkLayout L0(c.RCW, r_pad, n_rchunks, 0);
+  int stages = std::min(kb_per, 6);
+  while (stages > 1 && SplitkLayout(c.RCW, r_pad, n_rchunks, stages).total + 1024 > kSmemMax) --stages;
+  const SplitkLayout L(c.RCW, r_pad, n_rchunks, stages);
+  if (L.total + 1024 > kSmemMax) return false;
+  c.smem = L.total + 1024;
+  SplitkArgs& a = c.args;
+  std::memset(&a, 0, sizeof(a));
+  a.M = int32_t(M);
+  a.N = int32_t(N);
+  a.K = int32_t(K);
+  a.r_pad = r_pad;
+  a.n_rchunks = n_rchunks;
+  a.stages = stages;
+  a.splits = S;
+  a.kb_per_split = kb_per;
+  a.num_n = int32_t((N + 127) / 128);
+  a.wait_limit_ns = kWaitLimitNs;
+  (void)L0;
+  return true;
+}
+
+template <int RCW>
+lora_status_t launch_splitk_t(const CUtensorMap* maps, const SplitkCfg& c, cudaStream_t st) {
+  auto kern = fused_splitk_kernel<RCW>;
+  if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
+  const unsigned tiles = unsigned(((c.args.M + 127) / 128) * c.args.num_n);
+  const dim3 cl(unsigned(c.args.splits), 1, 1);
+  return launch_ex("split-K forward", kern, dim3(unsigned(c.args.splits), tiles), dim3(192), c.smem, st, &cl, maps[0],
+                   maps[1], maps[2], maps[3], c.args);
+}
+
+lora_status_t launch_splitk(const CUtensorMap* maps, const SplitkCfg& c, cudaStream_t st) {
+  if (c.RCW == 16) return launch_splitk_t<16>(maps, c, st);
+  if (c.RCW == 32) return launch_splitk_t<32>(maps, c, st);
+  return launch_splitk_t<64>(maps, c, st);
+}
+
 // ----------------------------------------------------------- skinny GEMM ----
 
 struct SkinnyCfg {
@@ -700,6 +776,19 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
   if (M == 0) return LORA_OK;
+  {
+    SplitkCfg k;
+    if (pick_splitk(M, d_out, d_in, r, dev.sm_count, k)) {
+      k.args.scale = alpha / float(r);
+      k.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
+      CUtensorMap maps[4];
+      if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) || !make_map(&maps[1], W, d_in, d_out, d_in, 64, 128, 128) ||
+          !make_map(&maps[2], A, d_in, r, d_in, 64, uint32_t(k.args.r_pad), 128) ||
+          !make_map(&maps[3], B, r, d_out, r, k.RCW, 128, k.RCW * 2))
+        return LORA_ERR_CUDA;
+      return launch_splitk(maps, k, reinterpret_cast<cudaStream_t>(stream));
+    }
+  }
   FusedCfg c;
   if (!pick_fused(M, d_out, d_in, r, false, dev.sm_count, c)) return LORA_ERR_RANK;
   c.args.scale = alpha / float(r);

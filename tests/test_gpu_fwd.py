@@ -113,3 +113,45 @@ def test_fwd_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in
     ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
     ok, info = lora_tol_check(f64(Y), ref)
     assert ok, info
+
+
+# Split-K forward (few output tiles): the S CTAs of a cluster share one
+# 128 x 128 tile and reduce T and the base through distributed shared memory.
+SPLITK_SHAPES = [
+    (128, 4096, 4096, 16, 32.0),    # 32 tiles, S = 4
+    (100, 1000, 520, 24, 18.0),     # ragged M, N and K; r = 24 -> 32
+    (64, 2048, 256, 128, 96.0),     # largest rank: N = 128 + 128 in one MMA
+    (200, 3072, 136, 8, 6.0),       # r = 8 -> 16, N tail of 8 columns
+    (384, 1344, 1024, 40, 30.0),    # 21 K blocks over 2 splits (11 + 10); 64-wide rank chunk
+]
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,alpha", SPLITK_SHAPES)
+def test_fwd_splitk_matches_oracle_and_fused(gpu, monkeypatch, M, d_in, d_out, r, alpha):
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=M + d_out + r)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+    monkeypatch.setenv("LORA_B200_SPLITK", "1")
+    Y1 = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    Y1b = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    assert torch.equal(Y1, Y1b)            # fixed-order reduction: bitwise repeatable
+    ok, info = lora_tol_check(f64(Y1), ref)
+    assert ok, ("split-K", info)
+    monkeypatch.setenv("LORA_B200_SPLITK", "0")
+    Y0 = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    ok, info = lora_tol_check(f64(Y0), ref)
+    assert ok, ("one CTA per tile", info)
+    assert gpu.lora_get_device_status() == 0
+
+
+def test_fwd_splitk_zero_adapter_gives_base(gpu, monkeypatch):
+    """B = 0 and A = 0 both give the base product exactly (split-K path)."""
+    monkeypatch.setenv("LORA_B200_SPLITK", "1")
+    sh = WL.LayerShape(128, 2048, 512, 16, 32.0)
+    t = WL.make_layer_inputs(sh, seed=5)
+    Y_b0 = run_fwd(gpu, t["X"], t["W"], t["A"], torch.zeros_like(t["B"]), sh.alpha)
+    Y_a0 = run_fwd(gpu, t["X"], t["W"], torch.zeros_like(t["A"]), t["B"], sh.alpha)
+    assert torch.equal(Y_b0, Y_a0)
+    ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), np.zeros((512, 16)), sh.alpha)
+    ok, info = lora_tol_check(f64(Y_b0), ref)
+    assert ok, info
