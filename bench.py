@@ -440,6 +440,49 @@ def run_sweep(args):
     return 0
 
 
+def _graph_replay_us(fn, flush, n, calls=1):
+    """Median device time of one CUDA-graph replay of `calls` back-to-back
+    calls of fn (captured after warm-up), L2 flushed before each replay."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            fn()
+    med, p10, p90 = _time_events(g.replay, flush, n)
+    del g
+    return med / calls, p10 / calls, p90 / calls
+
+
+def run_tiny(args):
+    """The tiny forward (X[256,512], W[512,512], r = 16): launch-bound, so
+    reported per call as eager (through the Python binding), CUDA-graph
+    replay of one call, and graph replay of 20 back-to-back calls."""
+    import torch
+    import lora_linear_layer_b200 as L
+    sh = WL.TINY_FWD
+    t = WL.make_layer_inputs(sh, seed=0)
+    X, W, A, B = (t[k].cuda() for k in ("X", "W", "A", "B"))
+    Y = torch.empty((sh.M, sh.d_out), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    fn = lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha)  # noqa: E731
+    eager = _time_events(fn, flush, args.steps)
+    g1 = _graph_replay_us(fn, flush, args.steps)
+    g20 = _graph_replay_us(fn, flush, args.steps, calls=20)
+    F = flops_fwd(sh.M, sh.d_in, sh.d_out, sh.r)
+    print(json.dumps({"workload": sh.name, "us_per_call_eager": eager[0], "us_per_call_graph": g1[0],
+                      "us_per_call_graph_x20": g20[0], "tflops_graph_x20": F / g20[0] / 1e6,
+                      "p10_p90_eager": [eager[1], eager[2]], "l2": "flushed before each timed call or replay"}),
+          flush=True)
+    return 0
+
+
 def run_merge(args):
     """The 36-layer x 7-target adapter merge (r = 32): one batched
     restore-and-merge refresh from the pristine copies per cycle."""
@@ -460,8 +503,13 @@ def run_merge(args):
         nbytes += 4.0 * d_out * d_in + 2.0 * r * (d_in + d_out)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     med, p10, p90 = _time_events(lambda: L.lora_merge_batched(items, r, alpha), flush, args.steps)
+    batch = L.MergeBatch(items, r)          # descriptors built once, as in a refresh loop
+    p_med = _time_events(lambda: batch(alpha), flush, args.steps)[0]
+    g_med = _graph_replay_us(lambda: batch(alpha), flush, args.steps)[0]
     print(json.dumps({"workload": "merge 36 layers x 7 targets, hidden 2560, r=32", "matrices": len(items),
                       "ms_per_cycle": med / 1e3, "ms_p10": p10 / 1e3, "ms_p90": p90 / 1e3,
+                      "ms_per_cycle_prepared": p_med / 1e3, "gbs_prepared": nbytes / p_med / 1e3,
+                      "ms_per_cycle_graph": g_med / 1e3,
                       "gbs": nbytes / med / 1e3, "hbm_frac": nbytes / med / 1e3 / (BW / 1e9),
                       "bytes_per_cycle": nbytes, "peak": f"HBM copy {BW/1e9:.0f} GB/s ({src})",
                       "inputs": "seeded torch.randn on the device (timing only; parity in tests)"}), flush=True)
@@ -484,11 +532,14 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="time lora_fwd on every sweep point (one line each)")
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
     ap.add_argument("--merge", action="store_true", help="time the 252-matrix batched merge refresh")
+    ap.add_argument("--tiny", action="store_true", help="time the tiny forward (eager and CUDA-graph replay)")
     args = ap.parse_args()
     if args.sweep:
         return run_sweep(args)
     if args.merge:
         return run_merge(args)
+    if args.tiny:
+        return run_tiny(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

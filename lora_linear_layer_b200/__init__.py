@@ -191,18 +191,34 @@ def lora_merge(W_src, A, B, W_dst, alpha: float, stream=None) -> None:
     _raise(code, "lora_merge")
 
 
+class MergeBatch:
+    """A batched merge prepared once for fixed buffers: the tensors are
+    checked and the descriptor array is built here, and every call passes the
+    same array to ``lora_merge_batched``.  This fits the adapter refresh,
+    which re-merges the same (pristine, A, B, W_inf) buffers each cycle after
+    updating A and B in place.  The tensors must stay alive and in place."""
+
+    def __init__(self, items: Sequence[Tuple], r: int):
+        self.n = len(items)
+        self.r = int(r)
+        self._arr = (_MergeDesc * max(self.n, 1))()
+        self._keep = []
+        for i, (W_src, A, B, W_dst) in enumerate(items):
+            d_out, d_in = W_src.shape
+            for t, nm, s in ((W_src, "W_src", (d_out, d_in)), (A, "A", (self.r, d_in)), (B, "B", (d_out, self.r)),
+                             (W_dst, "W_dst", (d_out, d_in))):
+                _check_tensor(t, nm, s)
+            self._arr[i] = _MergeDesc(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in)
+            self._keep.append((W_src, A, B, W_dst))
+
+    def __call__(self, alpha: float, stream=None) -> None:
+        code = lib().lora_merge_batched(self._arr, self.n, self.r, float(alpha), _stream(stream))
+        _raise(code, "lora_merge_batched")
+
+
 def lora_merge_batched(items: Sequence[Tuple], r: int, alpha: float, stream=None) -> None:
     """Merge every (W_src, A, B, W_dst) of ``items`` (shared r, alpha)."""
-    n = len(items)
-    arr = (_MergeDesc * max(n, 1))()
-    for i, (W_src, A, B, W_dst) in enumerate(items):
-        d_out, d_in = W_src.shape
-        for t, nm, s in ((W_src, "W_src", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
-                         (W_dst, "W_dst", (d_out, d_in))):
-            _check_tensor(t, nm, s)
-        arr[i] = _MergeDesc(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in)
-    code = lib().lora_merge_batched(arr, n, int(r), float(alpha), _stream(stream))
-    _raise(code, "lora_merge_batched")
+    MergeBatch(items, r)(alpha, stream)
 
 
 def lora_restore(W_src, W_dst, stream=None) -> None:

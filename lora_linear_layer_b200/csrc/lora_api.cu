@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <utility>
 #include <vector>
 
@@ -123,8 +124,10 @@ CUtensorMapSwizzle swz_enum(uint32_t span_bytes) {
 
 // 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
 // row pitch `ld` elements, box {box_inner, box_outer}.  Encoded maps are
-// kept in a small per-thread cache keyed by every encoding input, so a
-// layer called again on the same buffers skips the driver call.
+// kept in a per-thread hash table keyed by every encoding input, so a layer
+// (or a batched merge of hundreds of matrices) called again on the same
+// buffers skips the driver call.  The table is emptied when it reaches
+// kMapCache entries.
 struct MapKey {
   const void* ptr;
   uint64_t inner, outer, ld;
@@ -134,22 +137,25 @@ struct MapKey {
            swz == o.swz;
   }
 };
-constexpr int kMapCache = 64;
-struct MapCache {
-  MapKey key[kMapCache];
-  CUtensorMap map[kMapCache];
-  int used = 0, next = 0;
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.ptr) * 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {k.inner, k.outer, k.ld, uint64_t(k.bi) << 32 | k.bo, uint64_t(k.swz)})
+      h = (h ^ v) * 0x100000001B3ull + (h >> 29);
+    return size_t(h);
+  }
 };
-thread_local MapCache t_maps;
+constexpr size_t kMapCache = 8192;
+thread_local std::unordered_map<MapKey, CUtensorMap, MapKeyHash> t_maps;
 
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
               uint32_t box_outer, uint32_t swz_span_bytes) {
   const MapKey k{ptr, inner, outer, ld, box_inner, box_outer, swz_span_bytes};
-  for (int i = 0; i < t_maps.used; ++i)
-    if (t_maps.key[i] == k) {
-      *m = t_maps.map[i];
-      return true;
-    }
+  const auto it = t_maps.find(k);
+  if (it != t_maps.end()) {
+    *m = it->second;
+    return true;
+  }
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -162,9 +168,8 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
                  (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
     return false;
   }
-  const int slot = t_maps.used < kMapCache ? t_maps.used++ : (t_maps.next++ % kMapCache);
-  t_maps.key[slot] = k;
-  t_maps.map[slot] = *m;
+  if (t_maps.size() >= kMapCache) t_maps.clear();
+  t_maps.emplace(k, *m);
   return true;
 }
 

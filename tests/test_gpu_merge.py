@@ -115,3 +115,29 @@ def test_batched_merge_matches_single_and_restore_cycles_bit_identical(gpu):
         a, b = WL.perturb_adapter(m["A"], m["B"], 0)
         gpu.lora_merge(pristine[i], dev(a), dev(b), W_inf[i], alpha)
         assert torch.equal(W_inf[i], first_state[i])
+
+
+def test_prepared_merge_batch_follows_in_place_adapter_updates(gpu):
+    """A MergeBatch built once re-reads A and B on every call: after the
+    adapters are updated in place it gives the same bits as a fresh merge."""
+    r, alpha = 16, 32.0
+    shapes = [(640, 512), (256, 1032), (1000, 264)]
+    pristine, Ad, Bd = [], [], []
+    for i, (d_out, d_in) in enumerate(shapes):
+        m = WL.make_merge_inputs(d_out, d_in, r, seed=70 + i)
+        pristine.append(dev(m["W"]))
+        Ad.append(dev(m["A"]))
+        Bd.append(dev(m["B"]))
+    W_inf = [torch.empty_like(p) for p in pristine]
+    batch = gpu.MergeBatch(list(zip(pristine, Ad, Bd, W_inf)), r)
+    for cycle in range(2):
+        for i in range(len(shapes)):
+            a, b = WL.perturb_adapter(Ad[i].cpu(), Bd[i].cpu(), cycle, seed=90 + i)
+            Ad[i].copy_(dev(a))
+            Bd[i].copy_(dev(b))
+        batch(alpha)
+        for i in range(len(shapes)):
+            ref = torch.empty_like(pristine[i])
+            gpu.lora_merge(pristine[i], Ad[i], Bd[i], ref, alpha)
+            assert torch.equal(W_inf[i], ref)
+    assert gpu.lora_get_device_status() == 0
