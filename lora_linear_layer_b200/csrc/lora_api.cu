@@ -92,6 +92,14 @@ EncodeTiledFn g_encode = nullptr;
 lora_status_t device_info(DeviceInfo& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  // The tensor-map encoder is a driver call and needs a current context.  A
+  // thread that has not used the runtime yet (PyTorch's autograd worker, for
+  // one) has none: cudaSetDevice makes the device's primary context current.
+  thread_local int t_ctx_dev = -1;
+  if (t_ctx_dev != dev) {
+    if (cudaSetDevice(dev) != cudaSuccess) return LORA_ERR_CUDA;
+    t_ctx_dev = dev;
+  }
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& d = g_dev[dev];
   if (!d.probed) {

@@ -1,0 +1,130 @@
+"""The fused LoRA layer as PyTorch operators with autograd, and a module.
+
+    Y = X W^T + s (X A^T) B^T,   s = alpha / r   (or an explicit scale)
+
+fastaf 0.1.0, "FWD kernel speedup" / "BWD kernel speedup": the layer and its
+backward for a frozen base weight W; section "torch.compile compatibility":
+each kernel is a torch.library custom op with a fake implementation, so the
+compiler traces through the layer without a graph break (checked with
+torch._dynamo.explain).  Here:
+
+* ``torch.ops.lora_b200.lora_linear(X, W, A, B, scale)`` runs ``lora_fwd``;
+* ``torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, scale)`` runs
+  ``lora_bwd`` and returns (dX, dA, dB);
+* both have fake (meta) implementations, so they trace under FakeTensorMode
+  and torch.compile without graph breaks, and the first is differentiable
+  in X, A and B through the second.  W is frozen: it gets no gradient.
+
+The scale is passed explicitly, so rsLoRA's alpha / sqrt(r) (unsloth fork
+commit log, scripts/benchmarks/qwen3_flex_inference.py: PEFT keeps the
+adapter's scaling, alpha / sqrt(r) under rsLoRA, in the module) is as easy
+to use as alpha / r.  The C ABI takes
+alpha and computes s = alpha / r in fp32; these operators pass
+alpha = scale * r, which gives s exactly when r is a power of two and within
+one fp32 rounding otherwise.
+
+Argument marshalling only: all arithmetic runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import lora_bwd, lora_bwd_workspace_size, lora_fwd
+
+_LIB = "lora_b200"
+
+
+def _check(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor) -> Tuple[int, int, int, int]:
+    if X.dim() != 2 or W.dim() != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError("lora_linear takes 2-D X [M, d_in], W [d_out, d_in], A [r, d_in], B [d_out, r]")
+    M, d_in = X.shape
+    d_out, r = B.shape
+    if tuple(W.shape) != (d_out, d_in) or tuple(A.shape) != (r, d_in):
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, W {tuple(W.shape)}, A {tuple(A.shape)}, "
+                         f"B {tuple(B.shape)}")
+    return M, d_in, d_out, r
+
+
+@torch.library.custom_op(f"{_LIB}::lora_linear", mutates_args=())
+def lora_linear(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, scale: float) -> torch.Tensor:
+    """Y = X W^T + scale (X A^T) B^T (bf16, 2-D, contiguous CUDA tensors)."""
+    M, d_in, d_out, r = _check(X, W, A, B)
+    Y = torch.empty((M, d_out), dtype=X.dtype, device=X.device)
+    lora_fwd(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), Y, scale * r)
+    return Y
+
+
+@lora_linear.register_fake
+def _lora_linear_fake(X, W, A, B, scale):
+    M, d_in, d_out, r = _check(X, W, A, B)
+    return X.new_empty((M, d_out))
+
+
+@torch.library.custom_op(f"{_LIB}::lora_linear_bwd", mutates_args=())
+def lora_linear_bwd(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, dY: torch.Tensor,
+                    scale: float) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(dX, dA, dB) of Y = X W^T + scale (X A^T) B^T for the gradient dY."""
+    M, d_in, d_out, r = _check(X, W, A, B)
+    dX = torch.empty((M, d_in), dtype=X.dtype, device=X.device)
+    dA = torch.empty((r, d_in), dtype=A.dtype, device=A.device)
+    dB = torch.empty((d_out, r), dtype=B.dtype, device=B.device)
+    ws = torch.empty(max(lora_bwd_workspace_size(M, d_in, d_out, r), 1), dtype=torch.uint8, device=X.device)
+    lora_bwd(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
+             scale * r, ws)
+    return dX, dA, dB
+
+
+@lora_linear_bwd.register_fake
+def _lora_linear_bwd_fake(X, W, A, B, dY, scale):
+    M, d_in, d_out, r = _check(X, W, A, B)
+    return X.new_empty((M, d_in)), A.new_empty((r, d_in)), B.new_empty((d_out, r))
+
+
+def _setup_context(ctx, inputs, output):
+    X, W, A, B, scale = inputs
+    if W.requires_grad:
+        raise RuntimeError("lora_linear: the base weight W is frozen and gets no gradient; "
+                           "call W.requires_grad_(False)")
+    ctx.save_for_backward(X, W, A, B)
+    ctx.scale = scale
+
+
+def _backward(ctx, dY):
+    X, W, A, B = ctx.saved_tensors
+    dX, dA, dB = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY.contiguous(), ctx.scale)
+    return (dX if ctx.needs_input_grad[0] else None, None, dA if ctx.needs_input_grad[2] else None,
+            dB if ctx.needs_input_grad[3] else None, None)
+
+
+lora_linear.register_autograd(_backward, setup_context=_setup_context)
+
+
+class LoRALinear(torch.nn.Module):
+    """A linear layer with a frozen base weight and a trainable rank-r adapter:
+    y = x W^T + s (x A^T) B^T over the last dimension of x (any leading
+    dimensions).  s = alpha / r, or alpha / sqrt(r) with ``rslora=True``.
+    A is initialised N(0, 1/d_in) (variance), B to zero (the adapter starts
+    as the identity map of the base layer); all parameters are bf16."""
+
+    def __init__(self, d_in: int, d_out: int, r: int, alpha: float, rslora: bool = False,
+                 device: Optional[torch.device] = None, generator: Optional[torch.Generator] = None):
+        super().__init__()
+        self.d_in, self.d_out, self.r, self.alpha = int(d_in), int(d_out), int(r), float(alpha)
+        self.scale = self.alpha / (math.sqrt(self.r) if rslora else self.r)
+        kw = dict(dtype=torch.bfloat16, device=device)
+        self.weight = torch.nn.Parameter(
+            (torch.randn(d_out, d_in, generator=generator) * d_in ** -0.5).to(**kw), requires_grad=False)
+        self.lora_A = torch.nn.Parameter((torch.randn(r, d_in, generator=generator) * d_in ** -0.5).to(**kw))
+        self.lora_B = torch.nn.Parameter(torch.zeros(d_out, r, **kw))
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        y = torch.ops.lora_b200.lora_linear(x.reshape(-1, self.d_in), self.weight, self.lora_A, self.lora_B,
+                                            self.scale)
+        return y.reshape(*lead, self.d_out)
+
+    def extra_repr(self) -> str:
+        return f"d_in={self.d_in}, d_out={self.d_out}, r={self.r}, scale={self.scale:g}"

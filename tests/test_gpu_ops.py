@@ -1,0 +1,85 @@
+"""The torch operators and LoRALinear on the GPU: values and gradients
+against the fp64 oracle, through autograd, under torch.compile (fullgraph,
+eager backend) and with the rsLoRA scale."""
+import math
+
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+from gpu_helpers import f64
+from tolerance import lora_tol_check
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(gpu, d_in, d_out, r, alpha, seed, rslora=False):
+    from lora_linear_layer_b200 import ops
+    g = torch.Generator().manual_seed(seed)
+    m = ops.LoRALinear(d_in, d_out, r, alpha, rslora=rslora, device="cuda", generator=g)
+    with torch.no_grad():   # a trained-looking adapter (B = 0 would hide the up-projection)
+        m.lora_B.copy_((torch.randn(d_out, r, generator=g) * 0.02).to(torch.bfloat16))
+    return m
+
+
+def _oracle(m, x2d, dy2d):
+    alpha_eff = m.scale * m.r          # the oracle's s = alpha / r
+    X, W, A, B, dY = (f64(t.detach().cpu()) for t in (x2d, m.weight, m.lora_A, m.lora_B, dy2d))
+    Y = O.lora_forward(X, W, A, B, alpha_eff)
+    dX, dA, dB = O.lora_backward(X, W, A, B, dY, alpha_eff)
+    return Y, dX, dA, dB
+
+
+def _check_all(m, x, y, dy):
+    Y, dX, dA, dB = _oracle(m, x.reshape(-1, m.d_in), dy.reshape(-1, m.d_out))
+    for got, ref, name in ((y.reshape(-1, m.d_out), Y, "Y"), (x.grad.reshape(-1, m.d_in), dX, "dX"),
+                           (m.lora_A.grad, dA, "dA"), (m.lora_B.grad, dB, "dB")):
+        ok, info = lora_tol_check(f64(got.detach().cpu()), ref)
+        assert ok, (name, info)
+
+
+@pytest.mark.parametrize("rslora", [False, True])
+def test_module_forward_backward_matches_oracle(gpu, rslora):
+    m = _layer(gpu, 520, 264, 24, 18.0, seed=1, rslora=rslora)
+    x = WL.make_layer_inputs(WL.LayerShape(3 * 100, 520, 264, 24, 18.0), seed=2)["X"].reshape(3, 100, 520)
+    x = x.cuda().requires_grad_(True)
+    dy = (torch.randn(3, 100, 264, generator=torch.Generator().manual_seed(3))).to(torch.bfloat16).cuda()
+    y = m(x)
+    y.backward(dy)
+    assert m.weight.grad is None
+    _check_all(m, x, y, dy)
+
+
+def test_compiled_fullgraph_equals_eager(gpu):
+    m = _layer(gpu, 1024, 512, 16, 32.0, seed=4)
+    x0 = WL.make_layer_inputs(WL.LayerShape(256, 1024, 512, 16, 32.0), seed=5)["X"].cuda()
+    dy = torch.randn(256, 512, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).cuda()
+
+    def step(mod, x):
+        x = x.clone().requires_grad_(True)
+        mod.zero_grad(set_to_none=True)
+        y = mod(x)
+        y.backward(dy)
+        return y.detach(), x.grad, mod.lora_A.grad.clone(), mod.lora_B.grad.clone()
+
+    eager = step(m, x0)
+    torch._dynamo.reset()
+    cm = torch.compile(m, backend="eager", fullgraph=True)
+    comp = step(cm, x0)
+    for a, b in zip(eager, comp):
+        assert torch.equal(a, b)        # the same kernels on the same inputs
+    x = x0.clone().requires_grad_(True)
+    m.zero_grad(set_to_none=True)
+    y = m(x)
+    y.backward(dy)
+    _check_all(m, x, y, dy)
+
+
+def test_opcheck_schema_and_fake(gpu):
+    t = WL.make_layer_inputs(WL.LayerShape(130, 256, 136, 8, 6.0), seed=7, with_dy=True)
+    X, W, A, B, dY = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    torch.library.opcheck(torch.ops.lora_b200.lora_linear.default, (X, W, A, B, 0.75),
+                          test_utils=("test_schema", "test_faketensor"))
+    torch.library.opcheck(torch.ops.lora_b200.lora_linear_bwd.default, (X, W, A, B, dY, 0.75),
+                          test_utils=("test_schema", "test_faketensor"))

@@ -1,0 +1,88 @@
+"""The torch operators of lora_linear_layer_b200.ops on CPU: registration,
+fake (meta) shapes, autograd wiring and a graph-break-free trace.  No GPU:
+the real kernels only run in the -m gpu tests."""
+import math
+
+import pytest
+import torch
+from torch._subclasses.fake_tensor import FakeTensorMode
+
+from lora_linear_layer_b200 import ops
+
+
+def _fake_inputs(M=32, d_in=64, d_out=48, r=8):
+    X = torch.empty(M, d_in, dtype=torch.bfloat16, device="cuda")
+    W = torch.empty(d_out, d_in, dtype=torch.bfloat16, device="cuda")
+    A = torch.empty(r, d_in, dtype=torch.bfloat16, device="cuda")
+    B = torch.empty(d_out, r, dtype=torch.bfloat16, device="cuda")
+    return X, W, A, B
+
+
+def test_ops_are_registered():
+    assert hasattr(torch.ops.lora_b200, "lora_linear")
+    assert hasattr(torch.ops.lora_b200, "lora_linear_bwd")
+
+
+def test_fake_shapes_forward_and_backward():
+    with FakeTensorMode():
+        X, W, A, B = _fake_inputs()
+        Y = torch.ops.lora_b200.lora_linear(X, W, A, B, 2.0)
+        assert Y.shape == (32, 48) and Y.dtype == torch.bfloat16 and Y.device.type == "cuda"
+        dX, dA, dB = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, Y, 2.0)
+        assert dX.shape == (32, 64) and dA.shape == (8, 64) and dB.shape == (48, 8)
+
+
+def test_fake_rejects_mismatched_shapes():
+    with FakeTensorMode():
+        X, W, A, B = _fake_inputs()
+        with pytest.raises(ValueError):
+            torch.ops.lora_b200.lora_linear(X, W, A[:, :32], B, 2.0)
+
+
+def test_autograd_graph_routes_to_the_backward_op():
+    """On meta tensors (the fake implementations) the backward of lora_linear
+    runs lora_linear_bwd and returns gradients for X, A, B only (W frozen)."""
+    X, W, A, B = (t.to("meta") for t in (torch.empty(32, 64), torch.empty(48, 64), torch.empty(8, 64),
+                                          torch.empty(48, 8)))
+    X, W, A, B = (t.to(torch.bfloat16) for t in (X, W, A, B))
+    X.requires_grad_(True)
+    A.requires_grad_(True)
+    B.requires_grad_(True)
+    Y = torch.ops.lora_b200.lora_linear(X, W, A, B, 2.0)
+    assert Y.grad_fn is not None
+    gX, gA, gB = torch.autograd.grad(Y.sum(), (X, A, B))
+    assert gX.shape == X.shape and gA.shape == A.shape and gB.shape == B.shape
+
+
+def test_trainable_base_weight_is_refused():
+    with FakeTensorMode():
+        X, W, A, B = _fake_inputs()
+        W.requires_grad_(True)
+        A.requires_grad_(True)
+        with pytest.raises(RuntimeError, match="frozen"):
+            torch.ops.lora_b200.lora_linear(X, W, A, B, 2.0)
+
+
+def test_module_scale_and_init():
+    m = ops.LoRALinear(64, 48, 16, 32.0)
+    assert m.scale == 2.0
+    assert ops.LoRALinear(64, 48, 16, 32.0, rslora=True).scale == 32.0 / math.sqrt(16)
+    assert not m.weight.requires_grad and m.lora_A.requires_grad and m.lora_B.requires_grad
+    assert torch.count_nonzero(m.lora_B) == 0      # the adapter starts as the identity of the base
+    assert m.weight.dtype == torch.bfloat16
+
+
+def test_dynamo_traces_without_graph_breaks():
+    """torch._dynamo.explain over a function that calls the operator (fake
+    tensors, so nothing runs on a GPU): one graph, no breaks."""
+    import torch._dynamo
+
+    def f(X, W, A, B):
+        return torch.ops.lora_b200.lora_linear(X, W, A, B, 2.0) * 2
+
+    with FakeTensorMode():
+        args = _fake_inputs()
+    torch._dynamo.reset()
+    ex = torch._dynamo.explain(f)(*args)
+    assert ex.graph_break_count == 0
+    assert ex.graph_count == 1
