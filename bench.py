@@ -483,6 +483,65 @@ def run_tiny(args):
     return 0
 
 
+def compare_shapes():
+    """The pages' benchmark grid (fastaf 0.1.0, "FWD kernel speedup": batch
+    {1, 4, 16} x seq {256, 1024} x d_model {512, 1024, 2048} x rank {8, 16},
+    alpha = 2r, square layers), then the attention-projection and MLP
+    up-projection workloads."""
+    out = []
+    for b in (1, 4, 16):
+        for seq in (256, 1024):
+            for d in (512, 1024, 2048):
+                for r in (8, 16):
+                    out.append(WL.LayerShape(b * seq, d, d, r, 2.0 * r, name=f"b{b}_s{seq}_d{d}_r{r}"))
+    return out + [WL.ATTN_PROJ, WL.MLP_UP]
+
+
+def run_compare(args):
+    """Unfused PyTorch LoRA (cuBLAS matmuls, the pages' six-launch forward and
+    its autograd backward with W frozen) against lora_fwd / lora_bwd: median
+    device time of each, L2 flushed before every call, and the speedup."""
+    import torch
+    import lora_linear_layer_b200 as L
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for sh in compare_shapes():
+        if args.sweep_filter and args.sweep_filter not in sh.name:
+            continue
+        t = WL.make_layer_inputs(sh, seed=0, with_dy=True)
+        X, W, A, B, dY = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+        s = sh.alpha / sh.r
+        Y = torch.empty((sh.M, sh.d_out), dtype=torch.bfloat16, device="cuda")
+        dX = torch.empty_like(X)
+        dA = torch.empty_like(A)
+        dB = torch.empty_like(B)
+        ws = torch.empty(max(1, L.lora_bwd_workspace_size(sh.M, sh.d_in, sh.d_out, sh.r)), dtype=torch.uint8,
+                         device="cuda")
+        Xg, Ag, Bg = (v.clone().requires_grad_(True) for v in (X, A, B))
+
+        def torch_fwd():
+            return X @ W.t() + (X @ A.t()) @ B.t() * s
+
+        def torch_bwd():
+            y = Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s
+            return torch.autograd.grad(y, (Xg, Ag, Bg), dY)
+
+        n = max(5, min(args.steps, 50))
+        tf = _time_events(torch_fwd, flush, n)[0]
+        of = _time_events(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n)[0]
+        # the unfused backward includes its forward (autograd needs the graph); time the
+        # forward alone and subtract it
+        tfb = _time_events(torch_bwd, flush, n)[0]
+        ob = _time_events(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n)[0]
+        tb = max(tfb - _time_events(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n)[0], 1e-3)
+        print(json.dumps({"point": sh.name, "M": sh.M, "d_in": sh.d_in, "d_out": sh.d_out, "r": sh.r,
+                          "torch_fwd_us": tf, "ours_fwd_us": of, "fwd_speedup": tf / of,
+                          "torch_bwd_us": tb, "ours_bwd_us": ob, "bwd_speedup": tb / ob,
+                          "torch": "unfused: X@W.T + (X@A.T)@B.T*s, autograd backward (W frozen)",
+                          "l2": "flushed before every call"}), flush=True)
+        del X, W, A, B, dY, Y, dX, dA, dB, ws, Xg, Ag, Bg
+    return 0
+
+
 def run_merge(args):
     """The 36-layer x 7-target adapter merge (r = 32): one batched
     restore-and-merge refresh from the pristine copies per cycle."""
@@ -533,6 +592,8 @@ def main():
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
     ap.add_argument("--merge", action="store_true", help="time the 252-matrix batched merge refresh")
     ap.add_argument("--tiny", action="store_true", help="time the tiny forward (eager and CUDA-graph replay)")
+    ap.add_argument("--compare", action="store_true",
+                    help="unfused PyTorch LoRA vs lora_fwd / lora_bwd on the pages' grid (speedup)")
     args = ap.parse_args()
     if args.sweep:
         return run_sweep(args)
@@ -540,6 +601,8 @@ def main():
         return run_merge(args)
     if args.tiny:
         return run_tiny(args)
+    if args.compare:
+        return run_compare(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -366,8 +366,17 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
     a.band_w = num_n;
   }
   a.n_bands = (num_n + a.band_w - 1) / a.band_w;
+  // Runs of 8 N tiles of one M block, dealt round-robin, when there are
+  // enough of them for 80% of the clusters: the clusters then walk the same W
+  // tiles at the same time and the operands they share stay in L2 (measured,
+  // same box: 8192x4096x4096 forward 202.8 -> 192.5 us, 16384x4096x14336
+  // forward 1708 -> 1450 us and backward 2854 -> ~1750 us).  Otherwise the
+  // contiguous ranges inside column bands.
+  constexpr int kRunL = 8;
+  const int64_t runs = int64_t(num_m) * ((num_n + kRunL - 1) / kRunL);
+  const int64_t clusters = sm_count / c.CG;
   const int ro = run_override();
-  a.run_l = ro >= 0 ? ro : 0;
+  a.run_l = ro >= 0 ? ro : (num_n >= kRunL && runs * 5 >= clusters * 4 ? kRunL : 0);
   a.wait_limit_ns = kWaitLimitNs;
   return true;
 }
