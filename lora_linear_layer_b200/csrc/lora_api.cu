@@ -366,17 +366,28 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
     a.band_w = num_n;
   }
   a.n_bands = (num_n + a.band_w - 1) / a.band_w;
-  // Runs of 8 N tiles of one M block, dealt round-robin, when there are
-  // enough of them for 80% of the clusters: the clusters then walk the same W
-  // tiles at the same time and the operands they share stay in L2 (measured,
-  // same box: 8192x4096x4096 forward 202.8 -> 192.5 us, 16384x4096x14336
-  // forward 1708 -> 1450 us and backward 2854 -> ~1750 us).  Otherwise the
-  // contiguous ranges inside column bands.
-  constexpr int kRunL = 8;
-  const int64_t runs = int64_t(num_m) * ((num_n + kRunL - 1) / kRunL);
+  // Runs of L N tiles of one M block, dealt round-robin: the clusters walk
+  // the same W tiles at the same time, so the operands they share stay in
+  // L2, and T is computed once per run.  L in [2, 8] minimises the modelled
+  // makespan ceil(runs / clusters) * (L + 0.5) (a T computation costs about
+  // half a tile), over runs that keep at least 80% of the clusters busy;
+  // ties go to the longer run (runs of 16 measured no faster than 8).  Without such a run length: contiguous ranges inside
+  // column bands.  (Measured, same box: 8192x4096x4096 forward 202.8 ->
+  // 192.5 us at L = 8; 16384x4096x14336 forward 1708 -> 1329 us at L = 7.)
   const int64_t clusters = sm_count / c.CG;
+  int best_l = 0;
+  double best_cost = 0.0;
+  for (int l = 2; l <= std::min(num_n, 8); ++l) {
+    const int64_t runs = int64_t(num_m) * ((num_n + l - 1) / l);
+    if (runs * 5 < clusters * 4) continue;
+    const double cost = double((runs + clusters - 1) / clusters) * (l + 0.5);
+    if (best_l == 0 || cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && l > best_l)) {
+      best_l = l;
+      best_cost = cost;
+    }
+  }
   const int ro = run_override();
-  a.run_l = ro >= 0 ? ro : (num_n >= kRunL && runs * 5 >= clusters * 4 ? kRunL : 0);
+  a.run_l = ro >= 0 ? ro : best_l;
   a.wait_limit_ns = kWaitLimitNs;
   return true;
 }
