@@ -40,8 +40,10 @@ UNIT = "TFLOP/s"
 WORKLOADS = {"attn_proj": WL.ATTN_PROJ, "mlp_up": WL.MLP_UP}
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the sources the forward kernel's DRAM traffic depends on (kernel and launch
+# configuration / schedule)
 KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
-                  "lora_linear_layer_b200/csrc/common.cuh")
+                  "lora_linear_layer_b200/csrc/common.cuh", "lora_linear_layer_b200/csrc/lora_api.cu")
 LAUNCHES_PER_STEP = 5   # fwd 1; bwd: T (+ B transpose), dX, dB + dA; merge 1
 
 
