@@ -544,6 +544,42 @@ def run_compare(args):
     return 0
 
 
+def run_grouped(args):
+    """The seven LoRA targets of one layer of the merge model (hidden 2560:
+    q, k, v, o, gate, up, down; r = 16) as independent forwards on a batch of
+    M tokens: seven lora_fwd calls against one lora_fwd_batched call, eager
+    and as CUDA-graph replay, L2 flushed before each timed call or replay."""
+    import torch
+    import lora_linear_layer_b200 as L
+    r, alpha = 16, 32.0
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    for M in (256, 1024, 2048):
+        items = []
+        F = 0.0
+        for i, s in enumerate(WL.merge_shapes(layers=1)):
+            t = WL.make_layer_inputs(WL.LayerShape(M, s["d_in"], s["d_out"], r, alpha), seed=i)
+            X, W, A, B = (t[k].cuda() for k in ("X", "W", "A", "B"))
+            items.append((X, W, A, B, torch.empty((M, s["d_out"]), dtype=torch.bfloat16, device="cuda")))
+            F += flops_fwd(M, s["d_in"], s["d_out"], r)
+
+        def separate():
+            for (X, W, A, B, Y) in items:
+                L.lora_fwd(X, W, A, B, Y, alpha)
+
+        def grouped():
+            L.lora_fwd_batched(items, alpha)
+
+        sep = _time_events(separate, flush, args.steps)[0]
+        grp = _time_events(grouped, flush, args.steps)[0]
+        sep_g = _graph_replay_us(separate, flush, args.steps)[0]
+        grp_g = _graph_replay_us(grouped, flush, args.steps)[0]
+        print(json.dumps({"workload": f"7 LoRA targets of one hidden-2560 layer, M={M}, r={r}", "problems": len(items),
+                          "separate_us": sep, "grouped_us": grp, "separate_graph_us": sep_g,
+                          "grouped_graph_us": grp_g, "grouped_tflops_graph": F / grp_g / 1e6,
+                          "l2": "flushed before each timed call or replay"}), flush=True)
+    return 0
+
+
 def run_merge(args):
     """The 36-layer x 7-target adapter merge (r = 32): one batched
     restore-and-merge refresh from the pristine copies per cycle."""
@@ -594,6 +630,8 @@ def main():
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
     ap.add_argument("--merge", action="store_true", help="time the 252-matrix batched merge refresh")
     ap.add_argument("--tiny", action="store_true", help="time the tiny forward (eager and CUDA-graph replay)")
+    ap.add_argument("--grouped", action="store_true",
+                    help="seven small forwards: separate lora_fwd calls vs one lora_fwd_batched")
     ap.add_argument("--compare", action="store_true",
                     help="unfused PyTorch LoRA vs lora_fwd / lora_bwd on the pages' grid (speedup)")
     args = ap.parse_args()
@@ -605,6 +643,8 @@ def main():
         return run_tiny(args)
     if args.compare:
         return run_compare(args)
+    if args.grouped:
+        return run_grouped(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -166,6 +166,34 @@ lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int3
                                  float alpha, void* stream);
 
 /*
+ * Grouped forward: n independent forwards sharing r and alpha in one launch,
+ * for the launch-bound regime of many small layers (fastaf 0.1.0, "FWD
+ * kernel speedup": below the overhead threshold, launch overhead dominates
+ * small batches; e.g. the q, k and v projections of one input, or the
+ * adapters of several requests).  Each entry is one lora_fwd problem with
+ * lora_fwd's rules (entries with M = 0 are skipped).  No entry's Y may
+ * overlap another entry's inputs or Y (LORA_ERR_ALIAS).  `descs` is a HOST
+ * array of n entries, read during the call.  A problem with at least four
+ * 128 x 128 output tiles per SM of the GPU runs as lora_fwd would; the
+ * others share split-K launches (up to 40 problems per launch, longest
+ * contraction first).  Results match lora_fwd within the forward tolerance
+ * (the accumulation order may differ).
+ */
+typedef struct {
+  const void* X;
+  const void* W;
+  const void* A;
+  const void* B;
+  void* Y;
+  int64_t M;
+  int64_t d_in;
+  int64_t d_out;
+} lora_fwd_desc_t;
+
+lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float alpha,
+                               void* stream);
+
+/*
  * Restore: W_dst <- W_src, a bit copy of n_elems bf16 values (the pristine
  * copy is only read).
  */

@@ -36,6 +36,11 @@ class LoraLibraryMissing(ImportError):
     pass
 
 
+class _FwdDesc(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("Y", ctypes.c_void_p), ("M", ctypes.c_int64), ("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64)]
+
+
 class _MergeDesc(ctypes.Structure):
     _fields_ = [("W_src", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
                 ("W_dst", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64)]
@@ -64,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.lora_status_string.argtypes = [ctypes.c_int]
         L.lora_fwd.restype = ctypes.c_int
         L.lora_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
+        L.lora_fwd_batched.restype = ctypes.c_int
+        L.lora_fwd_batched.argtypes = [ctypes.POINTER(_FwdDesc), i32, i32, f32, vp]
         L.lora_bwd_workspace_size.restype = sz
         L.lora_bwd_workspace_size.argtypes = [i64, i64, i64, i32]
         L.lora_bwd.restype = ctypes.c_int
@@ -140,6 +147,27 @@ def lora_fwd(X, W, A, B, Y, alpha: float, stream=None) -> None:
     code = lib().lora_fwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r,
                           float(alpha), _stream(stream))
     _raise(code, "lora_fwd")
+
+
+def lora_fwd_batched(items: Sequence[Tuple], alpha: float, stream=None) -> None:
+    """One launch for several independent forwards (X, W, A, B, Y) that share
+    the rank r and alpha (see include/lora.h)."""
+    n = len(items)
+    arr = (_FwdDesc * max(n, 1))()
+    r = None
+    for i, (X, W, A, B, Y) in enumerate(items):
+        M, d_in = X.shape
+        d_out, r_i = B.shape
+        if r is None:
+            r = r_i
+        elif r_i != r:
+            raise ValueError(f"lora_fwd_batched: every problem needs the same rank ({r} vs {r_i})")
+        for t, nm, sh in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                          (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
+            _check_tensor(t, nm, sh)
+        arr[i] = _FwdDesc(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out)
+    code = lib().lora_fwd_batched(arr, n, int(r or 8), float(alpha), _stream(stream))
+    _raise(code, "lora_fwd_batched")
 
 
 def lora_bwd_workspace_size(M: int, d_in: int, d_out: int, r: int) -> int:

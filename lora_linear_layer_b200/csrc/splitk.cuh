@@ -18,22 +18,38 @@
 //     base partials in split order, rounds once to bf16 and stores them.
 // Nothing goes through global memory but Y, no atomics are used, and the
 // result is bitwise repeatable for a given shape.
+// A launch carries a table of problems with the same rank and scale
+// (blockIdx.y runs over the tiles of all of them), so many small layers can
+// share one launch.
 #pragma once
 
 #include "common.cuh"
 
 namespace lora {
 
-struct SplitkArgs {
+// One output problem of a launch (a grouped launch carries several, all with
+// the same rank and scale).
+struct SplitkJob {
+  CUtensorMap p;            // X [M, d_in], box {64, 128}
+  CUtensorMap q;            // W [d_out, d_in], box {64, 128}
+  CUtensorMap u;            // A [r, d_in], box {64, r_pad}
+  CUtensorMap v;            // B [d_out, r], box {RCW, 128}
   int32_t M, N, K;          // Y is [M, N]; contraction length K
+  int32_t num_n;            // column tiles of 128
+  int32_t tile_begin;       // first tile (blockIdx.y) of this problem
+  int32_t kb_per_split;     // K blocks of 64 per split
+  __nv_bfloat16* out;       // [M, N] row-major
+};
+
+template <int NJ>
+struct SplitkTable {
+  SplitkJob job[NJ];
+  int32_t n_jobs;
   int32_t r_pad;            // rank rounded up to 16
   int32_t n_rchunks;        // r_pad / RCW rounded up
   int32_t stages;           // pipeline depth
   int32_t splits;           // cluster size S (gridDim.x)
-  int32_t kb_per_split;     // K blocks of 64 per split
-  int32_t num_n;            // column tiles of 128
   float scale;              // s = alpha / r
-  __nv_bfloat16* out;       // [M, N] row-major
   uint64_t wait_limit_ns;
 };
 
@@ -62,11 +78,8 @@ struct SplitkLayout {
   }
 };
 
-template <int RCW>
-__global__ void __launch_bounds__(192, 1)
-    fused_splitk_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                        const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
-                        const SplitkArgs a) {
+template <int RCW, int NJ>
+__global__ void __launch_bounds__(192, 1) fused_splitk_kernel(const __grid_constant__ SplitkTable<NJ> a) {
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
   constexpr uint32_t kRSpan = RCW * 2;  // bytes per swizzled rank row
@@ -91,12 +104,16 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int split = int(cluster_ctarank());
+  // this cluster's problem and tile
   const int tile = int(blockIdx.y);
-  const int m = tile / a.num_n;
-  const int n = tile % a.num_n;
-  const int nk_total = (a.K + 63) / 64;
-  const int kb0 = split * a.kb_per_split;
-  const int kb1 = imin(nk_total, kb0 + a.kb_per_split);
+  int jix = 0;
+  while (jix + 1 < a.n_jobs && tile >= a.job[jix + 1].tile_begin) ++jix;
+  const SplitkJob& jb = a.job[jix];
+  const int m = (tile - jb.tile_begin) / jb.num_n;
+  const int n = (tile - jb.tile_begin) % jb.num_n;
+  const int nk_total = (jb.K + 63) / 64;
+  const int kb0 = split * jb.kb_per_split;
+  const int kb1 = imin(nk_total, kb0 + jb.kb_per_split);
   const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
   const uint64_t lim = a.wait_limit_ns;
 
@@ -114,10 +131,10 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmP);
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmU);
-    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&jb.p);
+    tma_prefetch_desc(&jb.q);
+    tma_prefetch_desc(&jb.u);
+    tma_prefetch_desc(&jb.v);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), 256);
@@ -144,7 +161,7 @@ __global__ void __launch_bounds__(192, 1)
       if (split == 0) {  // rank-side operand of the up-projection (B rows of this tile)
         mbar_arrive_expect_tx(vfull, L.v_bytes);
         for (int c = 0; c < a.n_rchunks; ++c)
-          tma_load_2d(sbase + L.off_v + uint32_t(c) * (128u * kRSpan), &tmV, vfull, c * RCW, n * 128);
+          tma_load_2d(sbase + L.off_v + uint32_t(c) * (128u * kRSpan), &jb.v, vfull, c * RCW, n * 128);
       }
       int stage = 0;
       uint32_t phase = 0;
@@ -154,9 +171,9 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t fb = full_bar(stage);
         mbar_arrive_expect_tx(fb, L.p_bytes + L.q_bytes + L.u_bytes);
         const int k0 = kb * 64;
-        tma_load_2d(st, &tmP, fb, k0, m * 128);
-        tma_load_2d(st + L.p_bytes, &tmQ, fb, k0, n * 128);
-        tma_load_2d(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, 0);
+        tma_load_2d(st, &jb.p, fb, k0, m * 128);
+        tma_load_2d(st + L.p_bytes, &jb.q, fb, k0, n * 128);
+        tma_load_2d(st + L.p_bytes + L.q_bytes, &jb.u, fb, k0, 0);
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
       if (*abort_flag) settle_ns(200000);  // let copies in flight land
@@ -344,8 +361,8 @@ __global__ void __launch_bounds__(192, 1)
           }
         const int grow = m * 128 + r0 + task / 32;
         const int gcol = n * 128 + (task % 32) * 4;
-        if (grow < a.M && gcol < a.N)  // N % 8 == 0: the 4 columns are all in or all out
-          *reinterpret_cast<uint2*>(a.out + (size_t)grow * a.N + gcol) =
+        if (grow < jb.M && gcol < jb.N)  // N % 8 == 0: the 4 columns are all in or all out
+          *reinterpret_cast<uint2*>(jb.out + (size_t)grow * jb.N + gcol) =
               make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
       }
     }

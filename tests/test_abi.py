@@ -125,3 +125,29 @@ def test_binding_rejects_cpu_tensors_before_any_cuda_call(built_lib):
     X = torch.zeros(8, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         built_lib.lora_fwd(X, X, X[:8], X, X.clone(), 16.0)
+
+
+def test_fwd_batched_validation_before_any_cuda_call(built_lib):
+    """lora_fwd_batched checks every entry (lora_fwd's rules) and that no
+    entry's Y overlaps another entry's inputs or Y, before touching the GPU."""
+    L = built_lib
+    so = L.lib()
+
+    def call(entries, r=16, n=None):
+        arr = (L._FwdDesc * max(len(entries), 1))(*[L._FwdDesc(*e) for e in entries])
+        return L.STATUS[so.lora_fwd_batched(arr, len(entries) if n is None else n, r, 32.0, None)]
+
+    a = _ptrs(5, base=ALIGNED)
+    b = _ptrs(5, base=ALIGNED + (1 << 40))
+    ok_a = (*a, 256, 512, 512)
+    ok_b = (*b, 128, 1024, 256)
+    assert L.STATUS[so.lora_fwd_batched(None, 1, 16, 32.0, None)] == "LORA_ERR_NULL"
+    assert call([ok_a], n=-1) == "LORA_ERR_SHAPE"
+    assert call([ok_a, (*b, 128, 1020, 256)]) == "LORA_ERR_SHAPE"     # d_in % 8 != 0
+    assert call([ok_a, ok_b], r=12) == "LORA_ERR_RANK"
+    assert call([ok_a, (b[0], b[1], b[2], b[3], 0, 128, 1024, 256)]) == "LORA_ERR_NULL"
+    assert call([ok_a, (b[0] + 8, *b[1:], 128, 1024, 256)]) == "LORA_ERR_ALIGN"
+    # entry 1 writes its Y into entry 0's X
+    assert call([ok_a, (*b[:4], a[0] + 4096, 128, 1024, 256)]) == "LORA_ERR_ALIAS"
+    # two entries share one Y
+    assert call([ok_a, (*b[:4], a[4], 128, 1024, 256)]) == "LORA_ERR_ALIAS"

@@ -155,3 +155,47 @@ def test_fwd_splitk_zero_adapter_gives_base(gpu, monkeypatch):
     ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), np.zeros((512, 16)), sh.alpha)
     ok, info = lora_tol_check(f64(Y_b0), ref)
     assert ok, info
+
+
+def test_fwd_batched_matches_oracle_and_is_repeatable(gpu):
+    """One grouped launch over problems of different sizes (an empty one
+    included) with a shared rank; every Y against the oracle."""
+    r, alpha = 24, 18.0
+    # (4096, 512, 2560) has 640 tiles (over four per SM): it takes the lora_fwd path
+    shapes = [(300, 520, 264), (1, 64, 136), (0, 256, 128), (700, 1024, 512), (128, 4096, 1024), (64, 2560, 4096),
+              (2048, 512, 1280), (4096, 512, 2560)]
+    items, hosts = [], []
+    for i, (M, d_in, d_out) in enumerate(shapes):
+        t = WL.make_layer_inputs(WL.LayerShape(M, d_in, d_out, r, alpha), seed=100 + i)
+        X, W, A, B = (dev(t[k]) for k in ("X", "W", "A", "B"))
+        items.append((X, W, A, B, torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")))
+        hosts.append(t)
+    gpu.lora_fwd_batched(items, alpha)
+    first = [it[4].clone() for it in items]
+    gpu.lora_fwd_batched(items, alpha)
+    assert gpu.lora_get_device_status() == 0
+    for (X, W, A, B, Y), Y1, t in zip(items, first, hosts):
+        assert torch.equal(Y, Y1)
+        if Y.shape[0] == 0:
+            continue
+        ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+        ok, info = lora_tol_check(f64(Y.cpu()), ref)
+        assert ok, (tuple(X.shape), tuple(W.shape), info)
+
+
+def test_fwd_batched_more_problems_than_one_launch(gpu):
+    """45 problems: the call splits them over two launches (40 per launch)."""
+    r, alpha = 16, 32.0
+    items, hosts = [], []
+    for i in range(45):
+        M, d_in, d_out = 64 + 8 * (i % 5), 256 + 64 * (i % 3), 128 + 8 * (i % 7)
+        t = WL.make_layer_inputs(WL.LayerShape(M, d_in, d_out, r, alpha), seed=200 + i)
+        X, W, A, B = (dev(t[k]) for k in ("X", "W", "A", "B"))
+        items.append((X, W, A, B, torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")))
+        hosts.append(t)
+    gpu.lora_fwd_batched(items, alpha)
+    assert gpu.lora_get_device_status() == 0
+    for (X, W, A, B, Y), t in zip(items, hosts):
+        ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+        ok, info = lora_tol_check(f64(Y.cpu()), ref)
+        assert ok, info
