@@ -13,18 +13,19 @@
 // up-projections, scale and add; "BWD kernel speedup": the dX kernel.)
 //
 // Per output tile of (128 * CG) x BN:
-//   * the K loop streams P, Q (and, on the first tile of an M block, U)
-//     through a TMA -> shared-memory ring; one thread issues tcgen05.mma
-//     for the base product into a TMEM accumulator and, on that first tile,
-//     the N = r product T = P U^T into a second TMEM region;
+//   * the K loop streams P, Q (and, on the first tile a cluster takes from an
+//     M block, U) through a TMA -> shared-memory ring; one thread issues
+//     tcgen05.mma for the base product into a TMEM accumulator and, on that
+//     first tile, the N = r product T = P U^T into a second TMEM region;
 //   * four epilogue warps drain T, scale it by s in fp32, round to bf16 and
 //     write it into shared memory in the UMMA K-major swizzled layout (it
 //     never goes to global memory in the forward);
 //   * one more MMA pass (K = r) accumulates (sT) V^T onto the base
 //     accumulator; the epilogue rounds once to bf16 and writes OUT with
 //     TMA stores of 32 x 32 boxes staged in shared memory.
-// T is kept in shared memory and reused for every further tile of the same
-// M block the CTA processes.  Warp roles: warp 0 = TMA producer, warp 1 =
+// T is kept in shared memory and reused for every following tile of the
+// same M block (the schedule gives a cluster runs of consecutive N tiles of
+// one M block).  Warp roles: warp 0 = TMA producer, warp 1 =
 // MMA issuer and TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes
 // 32*(w%4)...).
 //
