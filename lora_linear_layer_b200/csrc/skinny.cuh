@@ -221,14 +221,15 @@ __global__ void __launch_bounds__(192, 1)
 
   uint8_t* const red = gbase;  // fp32 partial rows (reuses the ring once the MMAs are done)
   if (warp >= 2) {
-    // side job while the K loop runs: transposed copy of B, one slice per
-    // row tile (split 0 only)
-    if (a.tr_src != nullptr && split == 0) {
-      const int per = (a.tr_rows + job_tiles - 1) / job_tiles;
-      const int n0 = bx * per;
-      const int n1 = imin(a.tr_rows, n0 + per);
-      for (int e = int(threadIdx.x) - 64; e < (n1 - n0) * a.tr_r; e += 128) {
-        const int n = n0 + e / a.tr_r, j = e % a.tr_r;
+    // side job while the K loop runs: transposed copy of B, spread over the
+    // epilogue threads of every CTA of the job; consecutive threads write
+    // consecutive elements of a row of B^T
+    if (a.tr_src != nullptr) {
+      const int nthr = job_tiles * a.splits * 128;
+      const int total = a.tr_rows * a.tr_r;
+#pragma unroll 4
+      for (int e = (bx * a.splits + split) * 128 + int(threadIdx.x) - 64; e < total; e += nthr) {
+        const int j = e / a.tr_rows, n = e % a.tr_rows;
         a.tr_dst[(size_t)j * a.tr_rows + n] = a.tr_src[(size_t)n * a.tr_r + j];
       }
     }
