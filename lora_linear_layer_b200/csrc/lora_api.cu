@@ -304,35 +304,35 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
   int fBN, fCG;
   tile_override(fBN, fCG);
-  // Preference order: CTA pairs with 256-wide tiles (least operand traffic
-  // per flop), then single CTAs, then 128-wide tiles; take the first that
-  // fits in shared memory and has at least one tile per cluster.
-  const int cands[4][2] = {{256, 2}, {256, 1}, {128, 2}, {128, 1}};
+  // Candidates in order of preference: 256-wide tiles first (least operand
+  // traffic per flop); CTA pairs first for long contractions, single CTAs
+  // first for K <= 1024 (measured faster there: 8192x512x512 16.4 vs
+  // 18.4 us, 4096x1024x1024 21.2 vs 22.6 us).  Take the first that fits in
+  // shared memory with tiles for at least 80% of its clusters (fewer,
+  // larger tiles beat more, smaller ones: 2048x2048x2048 28.7 us with 64
+  // pair tiles of 256 x 256 against 38.9 us with 128 of 256 x 128), else
+  // 128-wide single-CTA tiles (128-wide pairs measured slower in every
+  // case: 512x4096x4096 43.0 vs 41.0 us).  LORA_B200_FUSED_TILE can still
+  // force a 128-wide pair.
+  const bool short_k = K <= 1024;
+  const int cands[4][2] = {{256, short_k ? 1 : 2}, {256, short_k ? 2 : 1}, {128, 1}, {128, 2}};
   c.BN = 0;
-  for (int i = 0; i < 4; ++i) {
-    const int BN = cands[i][0], CG = cands[i][1];
-    if (fBN != 0 && (BN != fBN || CG != fCG)) continue;
-    const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks, 1);
-    if (S < (BN == 256 ? 3 : 2)) continue;
-    const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
-    const bool last = (i == 3) || fBN != 0;
-    if (!last && tiles < sm_count / CG) continue;
-    c.BN = BN;
-    c.CG = CG;
-    c.stages = S;
-    break;
-  }
-  if (c.BN == 0 && fBN != 0) {
-    // the requested configuration does not fit: choose as usual
-    for (int i = 0; i < 4 && c.BN == 0; ++i) {
+  for (int pass = 0; pass < 2 && c.BN == 0; ++pass) {  // pass 1 ignores an infeasible override
+    for (int i = 0; i < 4; ++i) {
       const int BN = cands[i][0], CG = cands[i][1];
+      const bool forced = pass == 0 && fBN != 0;
+      if (forced && (BN != fBN || CG != fCG)) continue;
+      if (!forced && i == 3) break;  // the 128-wide pair only when forced
       const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks, 1);
       if (S < (BN == 256 ? 3 : 2)) continue;
       const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
-      if (i < 3 && tiles < sm_count / CG) continue;
-      c.BN = BN;
-      c.CG = CG;
-      c.stages = S;
+      const bool fills = double(tiles) >= 0.8 * double(sm_count / CG);
+      if (forced || fills || i == 2) {
+        c.BN = BN;
+        c.CG = CG;
+        c.stages = S;
+        break;
+      }
     }
   }
   if (c.BN == 0) return false;
