@@ -42,6 +42,10 @@
  *   LORA_ERR_UNSUPPORTED_DEVICE.
  * - Calls on different streams may run concurrently; the library keeps no
  *   per-call state besides the per-device status word.
+ * - Kernels are launched with programmatic dependent launch: a kernel's
+ *   set-up may overlap the end of the previous kernel on the stream, but it
+ *   touches no global memory before that kernel has completed, so stream
+ *   order is kept (LORA_B200_PDL=0 in the environment turns this off).
  */
 #ifndef LORA_B200_H
 #define LORA_B200_H
@@ -81,6 +85,10 @@ const char* lora_status_string(lora_status_t status);
  * tensor memory beside the base product, scaled by s and rounded to bf16
  * (as an unfused bf16 X @ A.T would be), and fed to the up-projection,
  * which accumulates onto the base product before the single store of Y.
+ * When the output has few 128 x 128 tiles (small M or a small weight), the
+ * contraction is split over the CTAs of a thread-block cluster and the
+ * partial sums of T and of the base product are added in a fixed order
+ * through distributed shared memory (still on chip, no atomics).
  */
 lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y,
                        int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
