@@ -22,8 +22,11 @@ def _merge_check(t, W_out, r, alpha):
     return info
 
 
+# the last two give each persistent CTA several tiles, so the 2-stage (r = 128)
+# and 3-stage (r = 64) rings wrap around
 @pytest.mark.parametrize("d_out,d_in,r", [(96, 80, 32), (4096, 2560, 32), (1000, 520, 24), (2560, 9728, 32),
-                                          (136, 64, 8), (520, 1032, 64), (264, 384, 128)])
+                                          (136, 64, 8), (520, 1032, 64), (264, 384, 128),
+                                          (2048, 4096, 128), (4096, 2560, 64)])
 def test_merge_matches_oracle(gpu, d_out, d_in, r):
     alpha = 2.0 * r
     t = WL.make_merge_inputs(d_out, d_in, r, seed=d_out + d_in)
