@@ -260,9 +260,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   griddep_launch_dependents();
   griddep_wait();
 
-  // T accumulator placement: its own columns if two BN-wide accumulators
-  // and r_pad columns fit in 512, else it borrows the other accumulator.
-  const bool borrow = (2 * BN + a.r_pad) > 512;
+  // T placement.  128-wide single-CTA forward tiles fold T into the base
+  // product: U's rows follow Q's rows in the stage, so one MMA with
+  // N = BN + r_pad covers both, and each accumulator buffer is BN + r_pad
+  // columns wide with T in its last r_pad.  Otherwise T gets its own columns
+  // if two BN-wide accumulators and r_pad columns fit in 512, else it
+  // borrows the other accumulator.
+  constexpr bool kFold = CG == 1 && BN == 128 && !MN;
+  const uint32_t acc_stride = kFold ? uint32_t(BN + a.r_pad) : uint32_t(BN);
+  const bool borrow = !kFold && (2 * BN + a.r_pad) > 512;
   const int nk = (a.K + kBK - 1) / kBK;
   const uint64_t lim = a.wait_limit_ns;
   const int n_clusters = int(gridDim.x) / CG;
@@ -326,6 +332,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint32_t id_base = idesc_bf16(kBM * CG, BN, false, MN);
       const uint32_t id_t = idesc_bf16(kBM * CG, a.r_pad, false, false);
       const uint32_t id_up = idesc_bf16(kBM * CG, BN, false, MN);
+      const uint32_t id_fold = idesc_bf16(kBM * CG, BN + a.r_pad, false, false);
       TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
       uint32_t phase = 0, vcount = 0, ntt = 0, tcount = 0;
@@ -341,7 +348,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const uint32_t b = tcount & 1u;
         if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY, kClusterScope))
           break;
-        uint32_t t_col = 2u * BN;
+        uint32_t t_col = kFold ? b * acc_stride + BN : 2u * BN;
         if (ttile && borrow) {
           const uint32_t ob = b ^ 1u;
           if (!wait_bounded(accempty0 + 8u * ob, next_acc_parity(ob), abort_flag, lim, SITE_ACCEMPTY,
@@ -350,7 +357,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           t_col = ob * BN;
         }
         tc_fence_after();
-        const uint32_t d_acc = tmem + b * BN;
+        const uint32_t d_acc = tmem + b * acc_stride;
         // The K loop, instantiated twice: with the N = r products of T (first
         // tile of an M block) and without.  Keeping the plain loop free of
         // the second MMA stream, and issuing the T products after the base
@@ -368,9 +375,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               const uint64_t ad = smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
               const uint64_t bd = MN ? smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B)
                                      : smem_desc(sq + kk * 32u, 16u, 1024u, SWZ_128B);
-              G::mma(d_acc, ad, bd, id_base, (kb | kk) != 0);
+              G::mma(d_acc, ad, bd, (kFold && kWithT) ? id_fold : id_base, (kb | kk) != 0);
             }
-            if constexpr (kWithT) {
+            if constexpr (kWithT && !kFold) {
               const uint32_t su = sq + L.q_bytes;
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk)
@@ -432,7 +439,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (!warp_wait_bounded(tfull, ntt & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
         ++ntt;
         tc_fence_after();
-        const uint32_t t_col = borrow ? (b ^ 1u) * BN : 2u * BN;
+        const uint32_t t_col = kFold ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
         for (int col = 0; col < a.r_pad; col += 16) {
           uint32_t v[16];
           tmem_ld_x16(tmem + lane_base + t_col + uint32_t(col), v);
@@ -463,7 +470,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint32_t fpar = (b ? full_waits1++ : full_waits0++) & 1u;
       if (!warp_wait_bounded(accfull0 + 8u * b, fpar, abort_flag, lim, SITE_ACCFULL, kClusterScope)) break;
       tc_fence_after();
-      const uint32_t acc_col = b * BN;
+      const uint32_t acc_col = b * acc_stride;
       // Each 32-column chunk: TMEM -> registers -> bf16 -> this warp's
       // swizzled staging buffer -> one TMA store of 32 rows x 64 bytes
       // (rows past M and columns past N are clipped by the tensor map).
