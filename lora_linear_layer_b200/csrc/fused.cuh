@@ -1,18 +1,21 @@
-// fused.cuh - the fused LoRA GEMM: OUT = P Q^T + (s P U^T) V^T on tcgen05.
+// fused.cuh - the fused LoRA GEMMs on tcgen05.
 //
 // One kernel serves two steps of the layer:
-//   forward  (MN = false): P = X[M,d_in], Q = W[d_out,d_in], U = A[r,d_in],
-//                          V = B[d_out,r]; all operands K-major.
+//   forward  (MN = false): OUT = P Q^T + (s P U^T) V^T with P = X[M,d_in],
+//                          Q = W[d_out,d_in], U = A[r,d_in], V = B[d_out,r],
+//                          all operands K-major:
 //                          OUT = Y = X W^T + s (X A^T) B^T
-//   dX       (MN = true):  P = dY[M,d_out], Q(n,k) = W[k,n] and V(n,j) = A[j,n]
-//                          read MN-major, U = B^T[r,d_out] (a transposed copy
-//                          of B, K-major).
-//                          OUT = dX = dY W + (s dY B) A, and the bf16 dT = s dY B
-//                          is also written out (for dA).
+//   dX       (MN = true):  OUT = [P | U] [Q ; V] with P = dY[M,d_out],
+//                          Q = W[d_out,d_in], U = dT[M,r_pad] (the bf16
+//                          s dY B of the backward's first pass, K-major) and
+//                          V = A[r,d_in], read MN-major:
+//                          OUT = dX = dY W + dT A, one accumulator, one
+//                          rounding.  The rank-side product is just 1 or 2
+//                          more K blocks of the same K loop.
 // (fastaf 0.1.0, "FWD kernel speedup": base product plus the down- and
 // up-projections, scale and add; "BWD kernel speedup": the dX kernel.)
 //
-// Per output tile of (128 * CG) x BN:
+// Forward, per output tile of (128 * CG) x BN:
 //   * the K loop streams P, Q (and, on the first tile a cluster takes from an
 //     M block, U) through a TMA -> shared-memory ring; one thread issues
 //     tcgen05.mma for the base product into a TMEM accumulator and, on that
@@ -25,7 +28,8 @@
 //     TMA stores of 32 x 32 boxes staged in shared memory.
 // T is kept in shared memory and reused for every following tile of the
 // same M block (the schedule gives a cluster runs of consecutive N tiles of
-// one M block).  Warp roles: warp 0 = TMA producer, warp 1 =
+// one M block).  dX tiles have none of the T, U, V steps and take single-tile
+// runs.  Warp roles: warp 0 = TMA producer, warp 1 =
 // MMA issuer and TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes
 // 32*(w%4)...).
 //
@@ -56,9 +60,8 @@ struct FusedArgs {
   int32_t n_rchunks;        // r_pad / RCW rounded up
   int32_t stages;           // pipeline depth
   int32_t ep_bufs;          // output staging buffers per epilogue warp (1 or 2)
-  float scale;              // s = alpha / r
+  float scale;              // s = alpha / r (forward)
   __nv_bfloat16* out;       // [M, N] row-major, ld = N
-  __nv_bfloat16* t_out;     // optional [M, r_pad] bf16 copy of s*T (dT), or null
   int32_t num_m, num_n;     // tile counts (M tiles of 128 * CG rows)
   int32_t band_w, n_bands;  // column bands of the schedule
   int32_t run_l;            // 0: contiguous ranges; L > 0: runs of L N-tiles dealt round-robin
@@ -74,10 +77,11 @@ struct FusedLayout {
     const int bnc = BN / CG;            // Q / V rows held by this CTA
     p_bytes = kBM * kBK * 2;
     q_bytes = uint32_t(bnc * kBK * 2);
-    u_bytes = uint32_t((r_pad / CG) * 128);
+    // the dX form streams its rank-side operands through the ring
+    u_bytes = mn ? 0u : uint32_t((r_pad / CG) * 128);
     stage_bytes = p_bytes + q_bytes + u_bytes;
-    v_bytes = mn ? uint32_t((bnc / 64) * r_pad * 128) : uint32_t(n_rchunks * bnc * rcw * 2);
-    st_bytes = uint32_t(n_rchunks * kBM * rcw * 2);
+    v_bytes = mn ? 0u : uint32_t(n_rchunks * bnc * rcw * 2);
+    st_bytes = mn ? 0u : uint32_t(n_rchunks * kBM * rcw * 2);
     off_v = stage_bytes * stages;
     ep_bytes = 4u * uint32_t(ep_bufs) * kEpBufBytes;
     off_st = off_v + v_bytes;
@@ -192,6 +196,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(CG == 1 || CG == 2, "CG");
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
+  constexpr bool kQmn = MN;             // Q read MN-major
   using G = Group<CG>;
   constexpr int BNC = BN / CG;          // Q / V rows held by this CTA
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
@@ -268,8 +273,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   // borrows the other accumulator.
   constexpr bool kFold = CG == 1 && BN == 128 && !MN;
   const uint32_t acc_stride = kFold ? uint32_t(BN + a.r_pad) : uint32_t(BN);
-  const bool borrow = !kFold && (2 * BN + a.r_pad) > 512;
+  const bool borrow = !MN && !kFold && (2 * BN + a.r_pad) > 512;
   const int nk = (a.K + kBK - 1) / kBK;
+  // dX: K blocks [nk, nk_all) hold the rank-side product dT A
+  const int nk_all = MN ? nk + (a.r_pad + kBK - 1) / kBK : nk;
   const uint64_t lim = a.wait_limit_ns;
   const int n_clusters = int(gridDim.x) / CG;
   const int cluster_id = int(blockIdx.x) / CG;
@@ -283,12 +290,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       uint32_t phase = 0, vcount = 0;
       bool ok = true;
       while (ok && sch.next(m, n)) {
-        const bool ttile = (m != prev_m);
+        const bool ttile = !MN && (m != prev_m);
         prev_m = m;
         const uint32_t bytes = L.p_bytes + L.q_bytes + (ttile ? L.u_bytes : 0u);
         const int row0 = m * (kBM * CG) + int(rank) * kBM;
         const int qrow0 = n * BN + int(rank) * BNC;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk_all; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, lim, SITE_EMPTY, kClusterScope)) {
             ok = false;
             break;
@@ -296,40 +303,50 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const uint32_t st = sbase + uint32_t(stage) * L.stage_bytes;
           const uint32_t fb = G::leader_addr(full_bar(stage));
           if (leader) mbar_arrive_expect_tx(full_bar(stage), bytes * CG);
-          const int k0 = kb * kBK;
-          G::load(st, &tmP, fb, k0, row0);
-          if (!MN) {
-            G::load(st + L.p_bytes, &tmQ, fb, k0, qrow0);
+          // Each branch names its tensor maps directly: selecting between
+          // two kernel-parameter maps through a pointer makes every load take
+          // its descriptor from a runtime address, which measured ~10% slower
+          // (8192 x 4096 x 4096 dX: 181 vs 162 us without the tail block).
+          if (!MN || kb < nk) {
+            const int k0 = kb * kBK;
+            G::load(st, &tmP, fb, k0, row0);
+            if (!kQmn) {
+              G::load(st + L.p_bytes, &tmQ, fb, k0, qrow0);
+            } else {
+#pragma unroll
+              for (int i = 0; i < BNC / 64; ++i)
+                G::load(st + L.p_bytes + uint32_t(i) * 8192u, &tmQ, fb, qrow0 + 64 * i, k0);
+            }
+            if (ttile) G::load(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, int(rank) * u_rows);
           } else {
+            // dX tail: dT and A in place of dY and W (columns of dT and rows
+            // of A past r_pad come from the tensor maps' zero fill)
+            const int k0 = (kb - nk) * kBK;
+            G::load(st, &tmU, fb, k0, row0);
 #pragma unroll
             for (int i = 0; i < BNC / 64; ++i)
-              G::load(st + L.p_bytes + uint32_t(i) * 8192u, &tmQ, fb, qrow0 + 64 * i, k0);
+              G::load(st + L.p_bytes + uint32_t(i) * 8192u, &tmV, fb, qrow0 + 64 * i, k0);
           }
-          if (ttile) G::load(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, int(rank) * u_rows);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
+        if (MN) continue;
         // rank-side operand of the up-projection for this N tile
         if (!wait_bounded(vempty, (vcount & 1u) ^ 1u, abort_flag, lim, SITE_VEMPTY, kClusterScope)) break;
         ++vcount;
         const uint32_t sv = sbase + L.off_v;
         const uint32_t vb = G::leader_addr(vfull);
         if (leader) mbar_arrive_expect_tx(vfull, L.v_bytes * CG);
-        if (!MN) {
-          for (int c = 0; c < a.n_rchunks; ++c)
-            G::load(sv + uint32_t(c) * uint32_t(BNC * kRSpan), &tmV, vb, c * RCW, qrow0);
-        } else {
-#pragma unroll
-          for (int i = 0; i < BNC / 64; ++i)
-            G::load(sv + uint32_t(i) * uint32_t(a.r_pad * 128), &tmV, vb, qrow0 + 64 * i, 0);
-        }
+        for (int c = 0; c < a.n_rchunks; ++c)
+          G::load(sv + uint32_t(c) * uint32_t(BNC * kRSpan), &tmV, vb, c * RCW, qrow0);
       }
       if (*abort_flag) settle_ns(200000);  // let copies in flight land
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
     if (lane == 0 && leader) {
-      const uint32_t id_base = idesc_bf16(kBM * CG, BN, false, MN);
+      const uint32_t id_base = idesc_bf16(kBM * CG, BN, false, kQmn);
+      const uint32_t id_tail = idesc_bf16(kBM * CG, BN, false, true);  // dX: V = A is MN-major
       const uint32_t id_t = idesc_bf16(kBM * CG, a.r_pad, false, false);
       const uint32_t id_up = idesc_bf16(kBM * CG, BN, false, MN);
       const uint32_t id_fold = idesc_bf16(kBM * CG, BN + a.r_pad, false, false);
@@ -343,7 +360,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       };
       bool ok = true;
       while (ok && sch.next(m, n)) {
-        const bool ttile = (m != prev_m);
+        const bool ttile = !MN && (m != prev_m);
         prev_m = m;
         const uint32_t b = tcount & 1u;
         if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY, kClusterScope))
@@ -365,17 +382,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // the tensor pipe fed (measured: 242 -> 216 us on 8192x4096x4096).
         auto k_loop = [&](auto with_t) -> bool {
           constexpr bool kWithT = decltype(with_t)::value;
-          for (int kb = 0; kb < nk; ++kb) {
+          for (int kb = 0; kb < nk_all; ++kb) {
             if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL, kClusterScope)) return false;
             tc_fence_after();
             const uint32_t st = sbase + uint32_t(stage) * L.stage_bytes;
             const uint32_t sq = st + L.p_bytes;
+            if (!MN || kb < nk) {
+              // fully unrolled (a data-dependent trip count here measured
+              // 206 vs 185 us on the 8192 x 4096 x 4096 dX)
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
-              const uint64_t bd = MN ? smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B)
-                                     : smem_desc(sq + kk * 32u, 16u, 1024u, SWZ_128B);
-              G::mma(d_acc, ad, bd, (kFold && kWithT) ? id_fold : id_base, (kb | kk) != 0);
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t ad = smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
+                const uint64_t bd = kQmn ? smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B)
+                                         : smem_desc(sq + kk * 32u, 16u, 1024u, SWZ_128B);
+                G::mma(d_acc, ad, bd, (kFold && kWithT) ? id_fold : id_base, (kb | kk) != 0);
+              }
+            } else {
+              // dX tail block: A is MN-major; stop at r_pad (the rest is zero fill)
+              const int kk_n = imin(kBK / 16, (a.r_pad - (kb - nk) * kBK) / 16);
+              for (int kk = 0; kk < kk_n; ++kk)
+                G::mma(d_acc, smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B),
+                       smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B), id_tail, 1u);
             }
             if constexpr (kWithT && !kFold) {
               const uint32_t su = sq + L.q_bytes;
@@ -391,6 +418,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         };
         ok = ttile ? k_loop(std::true_type{}) : k_loop(std::false_type{});
         if (!ok) break;
+        if (MN) {
+          G::commit_all(accfull0 + 8u * b);
+          ++tcount;
+          continue;
+        }
         if (ttile) {
           G::commit_all(tfull);
           if (!wait_bounded(stfull, ntt & 1u, abort_flag, lim, SITE_STFULL, kClusterScope)) break;
@@ -405,8 +437,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const uint32_t c = uint32_t(kk * 16) / RCW;
           const uint32_t off = uint32_t((kk * 16) % RCW) * 2u;
           const uint64_t ad = smem_desc(s_t + c * uint32_t(kBM * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
-          const uint64_t bd = MN ? smem_desc(s_v + uint32_t(kk) * 2048u, uint32_t(a.r_pad) * 128u, 1024u, SWZ_128B)
-                                 : smem_desc(s_v + c * uint32_t(BNC * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
+          const uint64_t bd = smem_desc(s_v + c * uint32_t(BNC * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
           G::mma(d_acc, ad, bd, id_up, 1u);
         }
         G::commit_all(vempty);
@@ -431,10 +462,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const uint32_t ep_off = L.off_ep + uint32_t(q * a.ep_bufs) * kEpBufBytes;
     uint32_t epc = 0;  // output blocks staged so far
     while (sch.next(m, n)) {
-      const bool ttile = (m != prev_m);
+      const bool ttile = !MN && (m != prev_m);
       prev_m = m;
       const uint32_t b = tcount & 1u;
-      const int grow = m * (kBM * CG) + int(rank) * kBM + row;
       if (ttile) {
         if (!warp_wait_bounded(tfull, ntt & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
         ++ntt;
@@ -453,11 +483,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           uint8_t* chunk = st_ptr + c * (kBM * kRSpan);
           *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin, kRSpan)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin + 1, kRSpan)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          if (a.t_out != nullptr && n == 0 && grow < a.M) {
-            uint4* dst = reinterpret_cast<uint4*>(a.t_out + (size_t)grow * a.r_pad + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
         }
         fence_proxy_async_smem();
         tc_fence_before();

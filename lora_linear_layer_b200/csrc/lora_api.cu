@@ -374,10 +374,14 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   // ties go to the longer run (runs of 16 measured no faster than 8).  Without such a run length: contiguous ranges inside
   // column bands.  (Measured, same box: 8192x4096x4096 forward 202.8 ->
   // 192.5 us at L = 8; 16384x4096x14336 forward 1708 -> 1329 us at L = 7.)
+  // The dX form computes no T, so single-tile runs: the round-robin order
+  // alone keeps the tiles in flight on a few M blocks, and the makespan is
+  // ceil(tiles / clusters).  (Measured on 8192x4096x4096 without T products:
+  // runs of 8 on 64 clusters 186 us, single tiles on 74 clusters 168 us.)
   const int64_t clusters = sm_count / c.CG;
-  int best_l = 0;
+  int best_l = mn ? 1 : 0;
   double best_cost = 0.0;
-  for (int l = 2; l <= std::min(num_n, 8); ++l) {
+  for (int l = 2; !mn && l <= std::min(num_n, 8); ++l) {
     const int64_t runs = int64_t(num_m) * ((num_n + l - 1) / l);
     if (runs * 5 < clusters * 4) continue;
     const double cost = double((runs + clusters - 1) / clusters) * (l + 0.5);
@@ -443,6 +447,10 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
 
 template <bool MN, int CG>
 lora_status_t launch_fused_cg(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
+  if constexpr (MN) {  // the dX form has no rank chunks in shared memory
+    return c.BN == 256 ? launch_fused_t<256, true, 64, CG>(maps, c, sm_count, st)
+                       : launch_fused_t<128, true, 64, CG>(maps, c, sm_count, st);
+  }
   if (c.BN == 256) {
     if (c.RCW == 16) return launch_fused_t<256, MN, 16, CG>(maps, c, sm_count, st);
     if (c.RCW == 32) return launch_fused_t<256, MN, 32, CG>(maps, c, sm_count, st);
@@ -594,45 +602,65 @@ void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, int64_
   a.kb_per_split = kb_per;
   a.splits = splits;
   a.out_mode = out_mode;
+  a.r_mn = r_mn ? 1 : 0;
   a.scale = 1.0f;
   a.wait_limit_ns = kWaitLimitNs;
 }
 
-// One launch of one job (c1 == nullptr) or of two jobs with the same
-// template arguments, split count and shared-memory layout.
-template <bool P_MN, bool R_MN, int RCW>
+// Re-split a job's contraction into exactly `splits` ranges (a launch's
+// two jobs share one cluster shape); trailing ranges may be empty.
+void resplit_skinny(SkinnyCfg& c, int splits) {
+  const int nk = int((int64_t(c.args.K) + 63) / 64);
+  c.splits = splits;
+  c.args.splits = splits;
+  c.args.kb_per_split = std::max(1, (nk + splits - 1) / splits);
+}
+
+// One launch of one job (c1 == nullptr) or of two jobs with the same P
+// layout, RCW and split count; the launch takes the larger shared-memory
+// size of the two.
+template <bool P_MN, int RCW>
 lora_status_t launch_skinny_t(const CUtensorMap& p0, const CUtensorMap& r0, const SkinnyCfg& c0,
                               const CUtensorMap* p1, const CUtensorMap* r1, const SkinnyCfg* c1, cudaStream_t st) {
-  auto kern = skinny_kernel<P_MN, R_MN, RCW>;
-  if (!ensure_smem_attr(kern, c0.smem)) return LORA_ERR_CUDA;
+  auto kern = skinny_kernel<P_MN, RCW>;
+  const uint32_t smem = c1 != nullptr ? std::max(c0.smem, c1->smem) : c0.smem;
+  if (!ensure_smem_attr(kern, smem)) return LORA_ERR_CUDA;
   const int t0 = (c0.args.rows + 127) / 128;
   const int t1 = c1 != nullptr ? (c1->args.rows + 127) / 128 : 0;
   const dim3 cl(1, unsigned(c0.splits), 1);
-  return launch_ex("skinny", kern, dim3(unsigned(t0 + t1), unsigned(c0.splits)), dim3(192), c0.smem, st, &cl, p0, r0,
+  return launch_ex("skinny", kern, dim3(unsigned(t0 + t1), unsigned(c0.splits)), dim3(192), smem, st, &cl, p0, r0,
                    p1 != nullptr ? *p1 : p0, r1 != nullptr ? *r1 : r0, c0.args, c1 != nullptr ? c1->args : c0.args,
                    int32_t(t0));
 }
 
-template <bool P_MN, bool R_MN>
+template <bool P_MN>
 lora_status_t launch_skinny(const CUtensorMap& p0, const CUtensorMap& r0, const SkinnyCfg& c0, cudaStream_t st,
                             const CUtensorMap* p1 = nullptr, const CUtensorMap* r1 = nullptr,
                             const SkinnyCfg* c1 = nullptr) {
-  if (c0.RCW == 16) return launch_skinny_t<P_MN, R_MN, 16>(p0, r0, c0, p1, r1, c1, st);
-  if (c0.RCW == 32) return launch_skinny_t<P_MN, R_MN, 32>(p0, r0, c0, p1, r1, c1, st);
-  return launch_skinny_t<P_MN, R_MN, 64>(p0, r0, c0, p1, r1, c1, st);
+  if (c0.RCW == 16) return launch_skinny_t<P_MN, 16>(p0, r0, c0, p1, r1, c1, st);
+  if (c0.RCW == 32) return launch_skinny_t<P_MN, 32>(p0, r0, c0, p1, r1, c1, st);
+  return launch_skinny_t<P_MN, 64>(p0, r0, c0, p1, r1, c1, st);
 }
 
 // --------------------------------------------------------- bwd workspace ----
 
 struct BwdPlan {
-  SkinnyCfg t_cfg, db_cfg, da_cfg;
-  size_t off_t, off_dt, off_bt, total;
+  SkinnyCfg dt_cfg, t_cfg, db_cfg, da_cfg;
+  size_t off_t, off_dt, total;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
-  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, (M + 127) / 128, p.t_cfg);
+  // dT (contraction d_out) and T (contraction d_in) share the first launch
+  // and its split count, which the longer contraction sets for the row
+  // tiles of both jobs; the longer job goes first in the grid
+  const int64_t both_tiles = 2 * ((M + 127) / 128);
+  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, both_tiles, p.dt_cfg);
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, both_tiles, p.t_cfg);
+  const int s1 = d_out >= d_in ? p.dt_cfg.splits : p.t_cfg.splits;
+  resplit_skinny(p.dt_cfg, s1);
+  resplit_skinny(p.t_cfg, s1);
   // dB and dA share one launch, so they share its split count
   const int64_t dbda_tiles = (d_out + 127) / 128 + (d_in + 127) / 128;
   pick_skinny(d_out, M, r, true, OUT_ROWS_R, dbda_tiles, p.db_cfg);
@@ -641,8 +669,7 @@ void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
   const size_t tb = align256(size_t(M) * r_pad * 2);
   p.off_t = 0;                                         // T   bf16 [M, r_pad]
   p.off_dt = tb;                                       // dT  bf16 [M, r_pad]
-  p.off_bt = 2 * tb;                                   // B^T bf16 [r, d_out]
-  p.total = p.off_bt + align256(size_t(r) * size_t(d_out) * 2);
+  p.total = 2 * tb;
 }
 
 // -------------------------------------------------------- merge batching ----
@@ -761,6 +788,9 @@ const char* lora_status_string(lora_status_t s) {
   return "LORA_ERR_UNKNOWN";
 }
 
+static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in, int64_t d_out,
+                                    int32_t r, size_t workspace_bytes, size_t need);
+
 lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in,
                               int64_t d_out, int32_t r, size_t workspace_bytes) {
   if (op == 0) {
@@ -782,7 +812,20 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
       return LORA_ERR_ALIAS;
     return LORA_OK;
   }
-  if (op == 1) {
+  if (op == 1) return check_bwd_args(ptrs, n_ptrs, M, d_in, d_out, r, workspace_bytes,
+                                     lora_bwd_workspace_size(M, d_in, d_out, r));
+  if (op == 2) {
+    if (ptrs == nullptr || n_ptrs != 4) return LORA_ERR_NULL;
+    MergeItem it{ptrs[0], ptrs[1], ptrs[2], const_cast<void*>(ptrs[3]), d_out, d_in};
+    return check_merge_item(it, r);
+  }
+  return LORA_ERR_SHAPE;
+}
+
+// The backward's argument rules with `need` bytes of workspace required.
+static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in, int64_t d_out,
+                                    int32_t r, size_t workspace_bytes, size_t need) {
+  {
     // X, dY, dX (and the workspace) may be NULL only when M == 0; dA and dB
     // are always written (zeros when M == 0).
     if (ptrs == nullptr || n_ptrs != 9) return LORA_ERR_NULL;
@@ -794,8 +837,7 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
     if (s != LORA_OK) return s;
     for (int i = 0; i < 8; ++i)
       if (!aligned16(ptrs[i])) return LORA_ERR_ALIGN;
-    const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
-    if (need > 0) {
+    if (M > 0) {
       if (ptrs[8] == nullptr || workspace_bytes < need) return LORA_ERR_WORKSPACE;
       if ((reinterpret_cast<uintptr_t>(ptrs[8]) & 255u) != 0) return LORA_ERR_ALIGN;
     }
@@ -812,12 +854,6 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
     }
     return LORA_OK;
   }
-  if (op == 2) {
-    if (ptrs == nullptr || n_ptrs != 4) return LORA_ERR_NULL;
-    MergeItem it{ptrs[0], ptrs[1], ptrs[2], const_cast<void*>(ptrs[3]), d_out, d_in};
-    return check_merge_item(it, r);
-  }
-  return LORA_ERR_SHAPE;
 }
 
 lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
@@ -843,7 +879,6 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
   if (!pick_fused(M, d_out, d_in, r, false, dev.sm_count, c)) return LORA_ERR_RANK;
   c.args.scale = alpha / float(r);
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
-  c.args.t_out = nullptr;
   CUtensorMap maps[5];
   const uint32_t bnc = uint32_t(c.BN / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
@@ -943,11 +978,12 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
   return p.total;
 }
 
-lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
-                       void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+// The backward, with `need` bytes of workspace required.
+static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                             void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                             void* workspace, size_t workspace_bytes, size_t need, void* stream) {
   const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
-  lora_status_t s = lora_check_args(1, ptrs, 9, M, d_in, d_out, r, workspace_bytes);
+  lora_status_t s = check_bwd_args(ptrs, 9, M, d_in, d_out, r, workspace_bytes, need);
   if (s != LORA_OK) return s;
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
@@ -961,37 +997,40 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_t);
   __nv_bfloat16* dTws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_dt);
-  __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + p.off_bt);
   const float scale = alpha / float(r);
   const int r_pad = r_pad_of(r);
   const int rcw = rcw_of(r_pad);
 
-  // 1. T = X A^T (recomputed), bf16 [M, r_pad]; the same launch writes
-  //    B^T [r, d_out], the K-major rank operand of the dX step.
+
+  // 1. One launch, two jobs: dT = s dY B and T = X A^T (recomputed), each
+  //    bf16 [M, r_pad] with zero columns past r.  The longer contraction's
+  //    job takes the first row tiles of the grid, so it starts first.
   {
-    CUtensorMap mp, mr;
-    if (!make_map(&mp, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr, A, d_in, r, d_in, 64, r_pad, 128))
+    CUtensorMap mp_dt, mr_dt, mp_t, mr_t;
+    if (!make_map(&mp_dt, dY, d_out, M, d_out, 64, 128, 128) ||
+        !make_map(&mr_dt, B, r, d_out, r, rcw, 64, rcw * 2) ||
+        !make_map(&mp_t, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr_t, A, d_in, r, d_in, 64, r_pad, 128))
       return LORA_ERR_CUDA;
-    SkinnyCfg c = p.t_cfg;
-    c.args.out = Tws;
-    c.args.tr_src = reinterpret_cast<const __nv_bfloat16*>(B);
-    c.args.tr_dst = Bt;
-    c.args.tr_rows = int32_t(d_out);
-    c.args.tr_r = r;
-    if ((s = launch_skinny<false, false>(mp, mr, c, st)) != LORA_OK) return s;
+    SkinnyCfg cdt = p.dt_cfg;
+    cdt.args.out = dTws;
+    cdt.args.scale = scale;
+    SkinnyCfg ct = p.t_cfg;
+    ct.args.out = Tws;
+    s = d_out >= d_in ? launch_skinny<false>(mp_dt, mr_dt, cdt, st, &mp_t, &mr_t, &ct)
+                      : launch_skinny<false>(mp_t, mr_t, ct, st, &mp_dt, &mr_dt, &cdt);
+    if (s != LORA_OK) return s;
   }
-  // 2. dX = dY W + dT A with dT = s dY B (dT also written, bf16 [M, r_pad])
+  // 2. dX = dY W + dT A: one GEMM over the contraction [d_out | r_pad]
   {
     FusedCfg c;
     if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
-    c.args.scale = scale;
+    c.args.scale = 1.0f;
     c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
-    c.args.t_out = dTws;
     CUtensorMap maps[5];
     if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
         !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
-        !make_map(&maps[2], Bt, d_out, r, d_out, 64, uint32_t(r_pad / c.CG), 128) ||
-        !make_map(&maps[3], A, d_in, r, d_in, 64, r_pad, 128) ||
+        !make_map(&maps[2], dTws, r_pad, M, r_pad, 64, 128, 128) ||
+        !make_map(&maps[3], A, d_in, r, d_in, 64, 64, 128) ||
         !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
       return LORA_ERR_CUDA;
     if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
@@ -1010,9 +1049,16 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
     cb.args.scale = scale;
     SkinnyCfg ca = p.da_cfg;
     ca.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
-    if ((s = launch_skinny<true, true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
+    if ((s = launch_skinny<true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
   }
   return LORA_OK;
+}
+
+lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                       void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                 lora_bwd_workspace_size(M, d_in, d_out, r), stream);
 }
 
 lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
@@ -1178,6 +1224,6 @@ extern "C" lora_status_t lora_bwd_noalloc(const void* X, const void* W, const vo
     if ((s = device_info(dev)) != LORA_OK) return s;
     if ((s = noalloc_scratch_address(&scratch)) != LORA_OK) return s;
   }
-  return lora_bwd(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, scratch, need > 0 ? kNoAllocScratchBytes : 0,
-                  stream);
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+                 need, stream);
 }

@@ -3,6 +3,7 @@
 // The rank-sized products of the backward (fastaf 0.1.0, "BWD kernel
 // speedup": the dA and dB kernels, with the M reduction made parallel):
 //   T recompute:  P = X[M, d_in] (K-major),  R = A[r, d_in] (K-major)
+//   dT = s dY B:  P = dY[M, d_out] (K-major), R(j,k) = B[k, j] (MN)
 //   dB:           P(i,k) = dY[k, i] (MN),    R(j,k) = T[k, j] (MN)
 //   dA:           P(i,k) = X[k, i] (MN),     R(j,k) = dT[k, j] (MN)
 // i runs over 128-row tiles (UMMA M = 128) and the rank is the UMMA N.  The
@@ -13,8 +14,9 @@
 // split order, before one rounding to bf16.
 // Nothing goes through global memory and no atomics are used, so results
 // are bitwise repeatable for a given shape.
-// One launch can carry two independent jobs of the same form (dB and dA):
-// row tiles [0, x_split) of the grid run job 0, the rest job 1.
+// One launch can carry two independent jobs with the same P layout and
+// split count (dT and T; dB and dA): row tiles [0, x_split) of the grid run
+// job 0, the rest job 1.  R's layout is a per-job argument.
 #pragma once
 
 #include "common.cuh"
@@ -37,13 +39,9 @@ struct SkinnyArgs {
   int32_t kb_per_split;   // K blocks (of 64) per split
   int32_t splits;         // gridDim.y; the cluster size when > 1
   int32_t out_mode;       // SkinnyOut
+  int32_t r_mn;           // R is read MN-major (rank contiguous) rather than K-major
   float scale;            // applied to the reduced fp32 sum before rounding
   __nv_bfloat16* out;
-  // optional side job of the split-0 CTAs: Bt[j, n] = B[n, j] for n < tr_rows,
-  // j < tr_r (the transposed copy of B that the dX step reads)
-  const __nv_bfloat16* tr_src;
-  __nv_bfloat16* tr_dst;
-  int32_t tr_rows, tr_r;
   uint64_t wait_limit_ns;
 };
 
@@ -70,17 +68,14 @@ __host__ __device__ inline uint32_t tmem_cols_for(int r_pad) {
   return c;
 }
 
-template <bool P_MN, bool R_MN, int RCW>
+template <bool P_MN, int RCW>
 __global__ void __launch_bounds__(192, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmP0, const __grid_constant__ CUtensorMap tmR0,
                   const __grid_constant__ CUtensorMap tmP1, const __grid_constant__ CUtensorMap tmR1,
                   const __grid_constant__ SkinnyArgs a0, const __grid_constant__ SkinnyArgs a1, const int32_t x_split) {
   const bool second = int(blockIdx.x) >= x_split;
   const SkinnyArgs& a = second ? a1 : a0;
-  const CUtensorMap* const tmP = second ? &tmP1 : &tmP0;
-  const CUtensorMap* const tmR = second ? &tmR1 : &tmR0;
   const int bx = second ? int(blockIdx.x) - x_split : int(blockIdx.x);   // row tile within the job
-  const int job_tiles = second ? int(gridDim.x) - x_split : x_split;
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
   constexpr uint32_t kRSpan = RCW * 2;
 
@@ -88,7 +83,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (sbase - raw);
-  const SkinnyLayout L(R_MN, RCW, a.r_pad, a.n_rchunks, a.stages);
+  const bool r_mn = a.r_mn != 0;
+  const SkinnyLayout L(r_mn, RCW, a.r_pad, a.n_rchunks, a.stages);
   const int S = a.stages;
   const uint32_t bar0 = sbase + L.off_bar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -135,7 +131,11 @@ __global__ void __launch_bounds__(192, 1)
   const uint64_t lim = a.wait_limit_ns;
 
   if (warp == 0) {
-    if (lane == 0) {
+    // The loop is instantiated once per job with that job's tensor maps
+    // named directly: a map chosen through a runtime pointer would make
+    // every load take its descriptor from a runtime address (measured
+    // ~10% slower on the fused kernel).
+    auto produce = [&](const CUtensorMap& tmP, const CUtensorMap& tmR) {
       int stage = 0;
       uint32_t phase = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -145,25 +145,29 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(fb, L.stage_bytes);
         const int k0 = kb * 64;
         if (!P_MN) {
-          tma_load_2d(st, tmP, fb, k0, i0);
+          tma_load_2d(st, &tmP, fb, k0, i0);
         } else {
-          tma_load_2d(st, tmP, fb, i0, k0);
-          tma_load_2d(st + 8192u, tmP, fb, i0 + 64, k0);
+          tma_load_2d(st, &tmP, fb, i0, k0);
+          tma_load_2d(st + 8192u, &tmP, fb, i0 + 64, k0);
         }
         const uint32_t sr = st + L.p_bytes;
-        if (!R_MN) {
-          tma_load_2d(sr, tmR, fb, k0, 0);
+        if (!r_mn) {
+          tma_load_2d(sr, &tmR, fb, k0, 0);
         } else {
           for (int c = 0; c < a.n_rchunks; ++c)
-            tma_load_2d(sr + uint32_t(c) * (64u * kRSpan), tmR, fb, c * RCW, k0);
+            tma_load_2d(sr + uint32_t(c) * (64u * kRSpan), &tmR, fb, c * RCW, k0);
         }
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
+    };
+    if (lane == 0) {
+      if (second) produce(tmP1, tmR1);
+      else produce(tmP0, tmR0);
       if (*abort_flag) settle_ns(200000);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, a.r_pad, P_MN, R_MN);
+      const uint32_t idesc = idesc_bf16(128, a.r_pad, P_MN, r_mn);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = P_MN ? smem_desc(st + kk * 2048u, 8192u, 1024u, SWZ_128B)
                                    : smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B);
-          const uint64_t bd = R_MN ? smem_desc(sr + kk * (16u * kRSpan), 64u * kRSpan, 8u * kRSpan, kRSwz)
+          const uint64_t bd = r_mn ? smem_desc(sr + kk * (16u * kRSpan), 64u * kRSpan, 8u * kRSpan, kRSwz)
                                    : smem_desc(sr + kk * 32u, 16u, 1024u, SWZ_128B);
           umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0);
         }
@@ -221,18 +225,6 @@ __global__ void __launch_bounds__(192, 1)
 
   uint8_t* const red = gbase;  // fp32 partial rows (reuses the ring once the MMAs are done)
   if (warp >= 2) {
-    // side job while the K loop runs: transposed copy of B, spread over the
-    // epilogue threads of every CTA of the job; consecutive threads write
-    // consecutive elements of a row of B^T
-    if (a.tr_src != nullptr) {
-      const int nthr = job_tiles * a.splits * 128;
-      const int total = a.tr_rows * a.tr_r;
-#pragma unroll 4
-      for (int e = (bx * a.splits + split) * 128 + int(threadIdx.x) - 64; e < total; e += nthr) {
-        const int j = e / a.tr_rows, n = e % a.tr_rows;
-        a.tr_dst[(size_t)j * a.tr_rows + n] = a.tr_src[(size_t)n * a.tr_r + j];
-      }
-    }
     bool have = true;
     if (nkb > 0) {
       have = warp_wait_bounded(accfull, 0u, abort_flag, lim, SITE_ACCFULL);

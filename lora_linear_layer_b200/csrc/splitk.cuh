@@ -107,8 +107,11 @@ __global__ void __launch_bounds__(192, 1) fused_splitk_kernel(const __grid_const
   // this cluster's problem and tile
   const int tile = int(blockIdx.y);
   int jix = 0;
-  while (jix + 1 < a.n_jobs && tile >= a.job[jix + 1].tile_begin) ++jix;
-  const SplitkJob& jb = a.job[jix];
+  if constexpr (NJ > 1)
+    while (jix + 1 < a.n_jobs && tile >= a.job[jix + 1].tile_begin) ++jix;
+  // with one job the index is a compile-time 0, so its tensor maps are
+  // named directly rather than through a runtime address
+  const SplitkJob& jb = a.job[NJ > 1 ? jix : 0];
   const int m = (tile - jb.tile_begin) / jb.num_n;
   const int n = (tile - jb.tile_begin) % jb.num_n;
   const int nk_total = (jb.K + 63) / 64;
