@@ -96,8 +96,8 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
 
 /*
  * Bytes of device scratch lora_bwd needs for this shape (0 when M == 0).
- * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16) and a
- * transposed copy of B, bf16 [r, d_out].
+ * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16), each at a
+ * 256-byte aligned offset.
  */
 size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r);
 
@@ -106,7 +106,9 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
  *   dX[M, d_in]  = dY W + dT A       (bf16)
  *   dA[r, d_in]  = dT^T X            (bf16, reduced over M in fp32)
  *   dB[d_out, r] = s dY^T T          (bf16, reduced over M in fp32)
- * with T = X A^T recomputed and dT = s dY B (rounded to bf16 on chip).
+ * with T = X A^T recomputed and dT = s dY B, both rounded to bf16 and kept
+ * in the workspace by a first launch; dX is then one product over the
+ * contraction [d_out | r], dY W + dT A, rounded once.
  * `workspace` is caller-owned device memory of at least
  * lora_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on
  * entry do not matter and are clobbered.  Results are bitwise repeatable:
