@@ -71,7 +71,7 @@ struct FusedArgs {
 // Byte sizes / offsets of one CTA's shared-memory carve-up (host and device).
 struct FusedLayout {
   uint32_t p_bytes, q_bytes, u_bytes, stage_bytes, v_bytes, st_bytes, ep_bytes;
-  uint32_t off_v, off_st, off_ep, off_bar, total;
+  uint32_t off_st, off_ep, off_bar, total;
   __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages,
                                   int ep_bufs) {
     const int bnc = BN / CG;            // Q / V rows held by this CTA
@@ -80,11 +80,13 @@ struct FusedLayout {
     // the dX form streams its rank-side operands through the ring
     u_bytes = mn ? 0u : uint32_t((r_pad / CG) * 128);
     stage_bytes = p_bytes + q_bytes + u_bytes;
+    // V (the up-projection's rank-side operand of one N tile) travels
+    // through the ring as one more stage per tile: all its chunks fit in a
+    // stage's P and Q slots (v_bytes <= p_bytes + q_bytes for r_pad <= 128)
     v_bytes = mn ? 0u : uint32_t(n_rchunks * bnc * rcw * 2);
     st_bytes = mn ? 0u : uint32_t(n_rchunks * kBM * rcw * 2);
-    off_v = stage_bytes * stages;
     ep_bytes = 4u * uint32_t(ep_bufs) * kEpBufBytes;
-    off_st = off_v + v_bytes;
+    off_st = stage_bytes * stages;
     off_ep = off_st + st_bytes;
     off_bar = off_ep + ep_bytes;
     total = off_bar + 256;
@@ -211,18 +213,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const FusedLayout L(BN, CG, MN, RCW, a.r_pad, a.n_rchunks, a.stages, a.ep_bufs);
   const int S = a.stages;
   const uint32_t bar0 = sbase + L.off_bar;
-  // barrier map (8 bytes each); full / vfull / accempty / stfull / drain
-  // are used on the even CTA only
+  // barrier map (8 bytes each); full / accempty / stfull / drain are used
+  // on the even CTA only
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-  const uint32_t vfull = bar0 + 8u * (2 * S + 0);
-  const uint32_t vempty = bar0 + 8u * (2 * S + 1);
-  const uint32_t accfull0 = bar0 + 8u * (2 * S + 2);   // +8*b
-  const uint32_t accempty0 = bar0 + 8u * (2 * S + 4);  // +8*b
-  const uint32_t tfull = bar0 + 8u * (2 * S + 6);
-  const uint32_t stfull = bar0 + 8u * (2 * S + 7);
-  const uint32_t drain = bar0 + 8u * (2 * S + 8);
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_bar + 8 * (2 * S + 9));
+  const uint32_t accfull0 = bar0 + 8u * (2 * S + 0);   // +8*b
+  const uint32_t accempty0 = bar0 + 8u * (2 * S + 2);  // +8*b
+  const uint32_t tfull = bar0 + 8u * (2 * S + 4);
+  const uint32_t stfull = bar0 + 8u * (2 * S + 5);
+  const uint32_t drain = bar0 + 8u * (2 * S + 6);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_bar + 8 * (2 * S + 7));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -235,8 +235,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(vfull, 1);
-    mbar_init(vempty, 1);
     mbar_init(accfull0, 1);
     mbar_init(accfull0 + 8, 1);
     mbar_init(accempty0, 4 * CG);
@@ -287,7 +285,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (lane == 0) {
       TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
-      uint32_t phase = 0, vcount = 0;
+      uint32_t phase = 0;
       bool ok = true;
       while (ok && sch.next(m, n)) {
         const bool ttile = !MN && (m != prev_m);
@@ -331,14 +329,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
         if (!ok) break;
         if (MN) continue;
-        // rank-side operand of the up-projection for this N tile
-        if (!wait_bounded(vempty, (vcount & 1u) ^ 1u, abort_flag, lim, SITE_VEMPTY, kClusterScope)) break;
-        ++vcount;
-        const uint32_t sv = sbase + L.off_v;
-        const uint32_t vb = G::leader_addr(vfull);
-        if (leader) mbar_arrive_expect_tx(vfull, L.v_bytes * CG);
+        // rank-side operand of the up-projection for this N tile: one more
+        // ring stage, its RCW-wide chunks side by side from the stage base
+        if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, lim, SITE_EMPTY, kClusterScope)) break;
+        const uint32_t sv = sbase + uint32_t(stage) * L.stage_bytes;
+        const uint32_t vb = G::leader_addr(full_bar(stage));
+        if (leader) mbar_arrive_expect_tx(full_bar(stage), L.v_bytes * CG);
         for (int c = 0; c < a.n_rchunks; ++c)
           G::load(sv + uint32_t(c) * uint32_t(BNC * kRSpan), &tmV, vb, c * RCW, qrow0);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
       }
       if (*abort_flag) settle_ns(200000);  // let copies in flight land
     }
@@ -352,7 +351,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint32_t id_fold = idesc_bf16(kBM * CG, BN + a.r_pad, false, false);
       TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
-      uint32_t phase = 0, vcount = 0, ntt = 0, tcount = 0;
+      uint32_t phase = 0, ntt = 0, tcount = 0;
       uint32_t acc_waits0 = 0u, acc_waits1 = 0u;  // completed waits per accumulator
       auto next_acc_parity = [&](uint32_t buf) {
         const uint32_t k = buf ? acc_waits1++ : acc_waits0++;
@@ -428,11 +427,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           if (!wait_bounded(stfull, ntt & 1u, abort_flag, lim, SITE_STFULL, kClusterScope)) break;
           ++ntt;
         }
-        if (!wait_bounded(vfull, vcount & 1u, abort_flag, lim, SITE_VFULL, kClusterScope)) break;
-        ++vcount;
+        if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL, kClusterScope)) break;
         tc_fence_after();
         const uint32_t s_t = sbase + L.off_st;
-        const uint32_t s_v = sbase + L.off_v;
+        const uint32_t s_v = sbase + uint32_t(stage) * L.stage_bytes;  // this tile's V stage
         for (int kk = 0; kk < a.r_pad / 16; ++kk) {
           const uint32_t c = uint32_t(kk * 16) / RCW;
           const uint32_t off = uint32_t((kk * 16) % RCW) * 2u;
@@ -440,7 +438,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const uint64_t bd = smem_desc(s_v + c * uint32_t(BNC * kRSpan) + off, 16u, 8u * kRSpan, kRSwz);
           G::mma(d_acc, ad, bd, id_up, 1u);
         }
-        G::commit_all(vempty);
+        G::commit_all(empty_bar(stage));
+        if (++stage == S) { stage = 0; phase ^= 1u; }
         G::commit_all(accfull0 + 8u * b);
         ++tcount;
       }
