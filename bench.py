@@ -264,8 +264,12 @@ def run_ours(args):
     X, W, A, B, dY = (host[k].cuda() for k in ("X", "W", "A", "B", "dY"))
     Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
     dX = torch.empty((M, d_in), dtype=torch.bfloat16, device="cuda")
-    dA = torch.empty((r, d_in), dtype=torch.bfloat16, device="cuda")
-    dB = torch.empty((d_out, r), dtype=torch.bfloat16, device="cuda")
+    # with several ranks the adapter gradients stay fp32 until they are summed
+    # (lora_bwd_ex with LORA_BWD_FP32_GRADS), so the exchange adds unrounded
+    # partials; on one GPU they are the layer's bf16 outputs
+    gdt = torch.float32 if world > 1 else torch.bfloat16
+    dA = torch.empty((r, d_in), dtype=gdt, device="cuda")
+    dB = torch.empty((d_out, r), dtype=gdt, device="cuda")
     Wm = torch.empty_like(W)
     ws = torch.empty(L.lora_bwd_workspace_size(M, d_in, d_out, r), dtype=torch.uint8, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -279,9 +283,11 @@ def run_ours(args):
         L.lora_fwd(Xb, W, A, B, Y, alpha, stream)
         if ev_f1 is not None:
             ev_f1.record(stream)
-        L.lora_bwd(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, stream)
         if world > 1:
-            dp.allreduce_adapter_grads(dA, dB)   # the data-parallel exchange (NCCL)
+            L.lora_bwd_ex(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, L.LORA_BWD_FP32_GRADS, stream)
+            dp.allreduce_adapter_grads(dA, dB)   # the data-parallel exchange (NCCL), fp32
+        else:
+            L.lora_bwd(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, stream)
         L.lora_merge(W, A, B, Wm, alpha, stream)
 
     warm = max(3, args.warmup)
@@ -328,7 +334,7 @@ def run_ours(args):
         out_dA = torch.empty_like(dA, device="cpu").pin_memory()
         out_dB = torch.empty_like(dB, device="cpu").pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        d2h = out_dA.numel() * 2 + out_dB.numel() * 2
+        d2h = out_dA.numel() * out_dA.element_size() + out_dB.numel() * out_dB.element_size()
         Ke = max(3, min(K, args.e2e_steps))
 
         # Two device buffers per input: while step i computes on one, a copy

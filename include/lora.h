@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define LORA_ABI_VERSION 1
+#define LORA_ABI_VERSION 2
 
 typedef enum {
   LORA_OK = 0,
@@ -69,7 +69,8 @@ typedef enum {
   LORA_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed */
   LORA_ERR_TIMEOUT = 7,            /* a kernel gave up on a bounded wait */
   LORA_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not sm_100 */
-  LORA_ERR_ALIAS = 9               /* an output overlaps an input */
+  LORA_ERR_ALIAS = 9,              /* an output overlaps an input */
+  LORA_ERR_FLAGS = 10              /* a flags argument has an unknown bit set */
 } lora_status_t;
 
 /* ABI version of the loaded library (LORA_ABI_VERSION it was built with). */
@@ -120,6 +121,25 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
                        const void* dY, void* dX, void* dA, void* dB,
                        int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Flags of lora_bwd_ex. */
+#define LORA_BWD_FP32_GRADS 1u /* dA and dB are fp32 (float) instead of bf16 */
+
+/*
+ * lora_bwd with flags.  flags == 0 is exactly lora_bwd.  With
+ * LORA_BWD_FP32_GRADS, dA[r, d_in] and dB[d_out, r] are fp32 buffers (same
+ * shapes and layouts, 4 bytes per element, 16-byte aligned) and receive the
+ * fp32 reductions over M before any rounding: each value is the one that
+ * lora_bwd rounds to bf16 (RNE), so rounding them gives lora_bwd's results
+ * bit for bit.  Meant for fp32 optimizer states and for summing per-rank
+ * partial gradients in fp32 before a single rounding (data parallelism).
+ * With M == 0 they are set to zero.  Other rules as lora_bwd; an unknown
+ * flag bit returns LORA_ERR_FLAGS before anything is launched.
+ */
+lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const void* B,
+                          const void* dY, void* dX, void* dA, void* dB,
+                          int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                          void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
 
 /*
  * Backward without a workspace argument (the pages describe no such entry

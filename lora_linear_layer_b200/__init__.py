@@ -21,8 +21,9 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lora.h")
 STATUS = {
     0: "LORA_OK", 1: "LORA_ERR_NULL", 2: "LORA_ERR_SHAPE", 3: "LORA_ERR_ALIGN",
     4: "LORA_ERR_RANK", 5: "LORA_ERR_WORKSPACE", 6: "LORA_ERR_CUDA",
-    7: "LORA_ERR_TIMEOUT", 8: "LORA_ERR_UNSUPPORTED_DEVICE", 9: "LORA_ERR_ALIAS",
+    7: "LORA_ERR_TIMEOUT", 8: "LORA_ERR_UNSUPPORTED_DEVICE", 9: "LORA_ERR_ALIAS", 10: "LORA_ERR_FLAGS",
 }
+LORA_BWD_FP32_GRADS = 1
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.lora_bwd_workspace_size.argtypes = [i64, i64, i64, i32]
         L.lora_bwd.restype = ctypes.c_int
         L.lora_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, vp]
+        L.lora_bwd_ex.restype = ctypes.c_int
+        L.lora_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, ctypes.c_uint32, vp]
         L.lora_bwd_noalloc.restype = ctypes.c_int
         L.lora_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
         L.lora_merge.restype = ctypes.c_int
@@ -189,6 +192,29 @@ def lora_bwd(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, stream=None) -
     code = lib().lora_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
                           M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, _stream(stream))
     _raise(code, "lora_bwd")
+
+
+def lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, flags: int = 0, stream=None) -> None:
+    """lora_bwd with flags (see include/lora.h).  With LORA_BWD_FP32_GRADS,
+    dA and dB are float32 tensors and receive the fp32 reductions that
+    lora_bwd would round to bf16."""
+    import torch
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r)), (dY, "dY", (M, d_out)), (dX, "dX", (M, d_in))):
+        _check_tensor(t, n, s)
+    gdt = torch.float32 if int(flags) & LORA_BWD_FP32_GRADS else torch.bfloat16
+    for t, n, s in ((dA, "dA", (r, d_in)), (dB, "dB", (d_out, r))):
+        if not isinstance(t, torch.Tensor) or t.dtype != gdt:
+            raise TypeError(f"{n} must be a {gdt} tensor with these flags")
+        if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != s:
+            raise ValueError(f"{n} must be a contiguous CUDA tensor of shape {s}")
+    ws_bytes = int(workspace.numel() * workspace.element_size())
+    code = lib().lora_bwd_ex(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
+                             M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, int(flags),
+                             _stream(stream))
+    _raise(code, "lora_bwd_ex")
 
 
 def lora_bwd_noalloc(X, W, A, B, dY, dX, dA, dB, alpha: float, stream=None) -> None:

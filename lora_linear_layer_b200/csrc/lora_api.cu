@@ -784,12 +784,13 @@ const char* lora_status_string(lora_status_t s) {
     case LORA_ERR_TIMEOUT: return "LORA_ERR_TIMEOUT: a kernel gave up on a bounded wait";
     case LORA_ERR_UNSUPPORTED_DEVICE: return "LORA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
     case LORA_ERR_ALIAS: return "LORA_ERR_ALIAS: an output overlaps an input";
+    case LORA_ERR_FLAGS: return "LORA_ERR_FLAGS: unknown bit in a flags argument";
   }
   return "LORA_ERR_UNKNOWN";
 }
 
 static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in, int64_t d_out,
-                                    int32_t r, size_t workspace_bytes, size_t need);
+                                    int32_t r, size_t workspace_bytes, size_t need, int grad_bytes = 2);
 
 lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in,
                               int64_t d_out, int32_t r, size_t workspace_bytes) {
@@ -813,7 +814,7 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
     return LORA_OK;
   }
   if (op == 1) return check_bwd_args(ptrs, n_ptrs, M, d_in, d_out, r, workspace_bytes,
-                                     lora_bwd_workspace_size(M, d_in, d_out, r));
+                                     lora_bwd_workspace_size(M, d_in, d_out, r), 2);
   if (op == 2) {
     if (ptrs == nullptr || n_ptrs != 4) return LORA_ERR_NULL;
     MergeItem it{ptrs[0], ptrs[1], ptrs[2], const_cast<void*>(ptrs[3]), d_out, d_in};
@@ -822,9 +823,10 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
   return LORA_ERR_SHAPE;
 }
 
-// The backward's argument rules with `need` bytes of workspace required.
+// The backward's argument rules with `need` bytes of workspace required and
+// dA, dB of `grad_bytes` per element.
 static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int64_t M, int64_t d_in, int64_t d_out,
-                                    int32_t r, size_t workspace_bytes, size_t need) {
+                                    int32_t r, size_t workspace_bytes, size_t need, int grad_bytes) {
   {
     // X, dY, dX (and the workspace) may be NULL only when M == 0; dA and dB
     // are always written (zeros when M == 0).
@@ -844,8 +846,9 @@ static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int
     const Range in[5] = {range_of(ptrs[0], uint64_t(M) * d_in * 2), range_of(ptrs[1], uint64_t(d_out) * d_in * 2),
                          range_of(ptrs[2], uint64_t(r) * d_in * 2), range_of(ptrs[3], uint64_t(d_out) * r * 2),
                          range_of(ptrs[4], uint64_t(M) * d_out * 2)};
-    const Range out[4] = {range_of(ptrs[5], uint64_t(M) * d_in * 2), range_of(ptrs[6], uint64_t(r) * d_in * 2),
-                          range_of(ptrs[7], uint64_t(d_out) * r * 2), range_of(ptrs[8], need)};
+    const Range out[4] = {range_of(ptrs[5], uint64_t(M) * d_in * 2),
+                          range_of(ptrs[6], uint64_t(r) * d_in * uint64_t(grad_bytes)),
+                          range_of(ptrs[7], uint64_t(d_out) * r * uint64_t(grad_bytes)), range_of(ptrs[8], need)};
     for (int o = 0; o < 4; ++o) {
       for (int i = 0; i < 5; ++i)
         if (overlaps(out[o], in[i])) return LORA_ERR_ALIAS;
@@ -978,19 +981,23 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
   return p.total;
 }
 
-// The backward, with `need` bytes of workspace required.
+// The backward, with `need` bytes of workspace required; `flags` as in
+// lora_bwd_ex.
 static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
                              void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
-                             void* workspace, size_t workspace_bytes, size_t need, void* stream) {
+                             void* workspace, size_t workspace_bytes, size_t need, uint32_t flags, void* stream) {
+  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
+  const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
+  const int gb = f32 ? 4 : 2;  // bytes per dA / dB element
   const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
-  lora_status_t s = check_bwd_args(ptrs, 9, M, d_in, d_out, r, workspace_bytes, need);
+  lora_status_t s = check_bwd_args(ptrs, 9, M, d_in, d_out, r, workspace_bytes, need, gb);
   if (s != LORA_OK) return s;
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (M == 0) {
-    if ((s = zero_bytes(dA, size_t(r) * d_in * 2, st)) != LORA_OK) return s;
-    return zero_bytes(dB, size_t(d_out) * r * 2, st);
+    if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
+    return zero_bytes(dB, size_t(d_out) * r * gb, st);
   }
   BwdPlan p;
   plan_bwd(M, d_in, d_out, r, p);
@@ -1047,8 +1054,10 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
     SkinnyCfg cb = p.db_cfg;
     cb.args.out = reinterpret_cast<__nv_bfloat16*>(dB);
     cb.args.scale = scale;
+    cb.args.out_f32 = f32 ? 1 : 0;
     SkinnyCfg ca = p.da_cfg;
     ca.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
+    ca.args.out_f32 = f32 ? 1 : 0;
     if ((s = launch_skinny<true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
   }
   return LORA_OK;
@@ -1058,7 +1067,14 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
                        void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                        void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
-                 lora_bwd_workspace_size(M, d_in, d_out, r), stream);
+                 lora_bwd_workspace_size(M, d_in, d_out, r), 0u, stream);
+}
+
+lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                          void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                          void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                 lora_bwd_workspace_size(M, d_in, d_out, r), flags, stream);
 }
 
 lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
@@ -1225,5 +1241,5 @@ extern "C" lora_status_t lora_bwd_noalloc(const void* X, const void* W, const vo
     if ((s = noalloc_scratch_address(&scratch)) != LORA_OK) return s;
   }
   return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, scratch, need > 0 ? kNoAllocScratchBytes : 0,
-                 need, stream);
+                 need, 0u, stream);
 }

@@ -40,8 +40,9 @@ struct SkinnyArgs {
   int32_t splits;         // gridDim.y; the cluster size when > 1
   int32_t out_mode;       // SkinnyOut
   int32_t r_mn;           // R is read MN-major (rank contiguous) rather than K-major
+  int32_t out_f32;        // OUT_ROWS_R / OUT_COLS_R: write fp32 (no rounding) instead of bf16
   float scale;            // applied to the reduced fp32 sum before rounding
-  __nv_bfloat16* out;
+  __nv_bfloat16* out;     // (a float* when out_f32)
   uint64_t wait_limit_ns;
 };
 
@@ -208,8 +209,16 @@ __global__ void __launch_bounds__(192, 1)
       dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     } else if (a.out_mode == OUT_ROWS_R) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {               // 8 values = 16 bytes, r % 8 == 0
+      for (int h = 0; h < 2; ++h) {               // 8 values, r % 8 == 0
         if (col0 + 8 * h >= a.r) break;
+        if (a.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + (size_t)gi * a.r + col0 + 8 * h);
+          dst[0] = make_float4(acc[8 * h] * a.scale, acc[8 * h + 1] * a.scale, acc[8 * h + 2] * a.scale,
+                               acc[8 * h + 3] * a.scale);
+          dst[1] = make_float4(acc[8 * h + 4] * a.scale, acc[8 * h + 5] * a.scale, acc[8 * h + 6] * a.scale,
+                               acc[8 * h + 7] * a.scale);
+          continue;
+        }
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -218,8 +227,12 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if (col0 + e < a.r) a.out[(size_t)(col0 + e) * a.rows + gi] = __float2bfloat16_rn(acc[e] * a.scale);
+      for (int e = 0; e < 16; ++e) {
+        if (col0 + e >= a.r) continue;
+        const size_t o = (size_t)(col0 + e) * a.rows + gi;
+        if (a.out_f32) reinterpret_cast<float*>(a.out)[o] = acc[e] * a.scale;
+        else a.out[o] = __float2bfloat16_rn(acc[e] * a.scale);
+      }
     }
   };
 
@@ -293,13 +306,22 @@ __global__ void __launch_bounds__(192, 1)
             *reinterpret_cast<uint2*>(a.out + (size_t)g * a.r_pad + j0) =
                 make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
           } else if (a.out_mode == OUT_ROWS_R) {
-            if (j0 < a.r)  // r % 8 == 0, so the 4 columns are all in or all out
-              *reinterpret_cast<uint2*>(a.out + (size_t)g * a.r + j0) =
-                  make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+            if (j0 < a.r) {  // r % 8 == 0, so the 4 columns are all in or all out
+              if (a.out_f32)
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + (size_t)g * a.r + j0) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+              else
+                *reinterpret_cast<uint2*>(a.out + (size_t)g * a.r + j0) =
+                    make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (j0 + e < a.r) a.out[(size_t)(j0 + e) * a.rows + g] = __float2bfloat16_rn(v[e]);
+            for (int e = 0; e < 4; ++e) {
+              if (j0 + e >= a.r) continue;
+              const size_t o = (size_t)(j0 + e) * a.rows + g;
+              if (a.out_f32) reinterpret_cast<float*>(a.out)[o] = v[e];
+              else a.out[o] = __float2bfloat16_rn(v[e]);
+            }
           }
         }
       }

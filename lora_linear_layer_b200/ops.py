@@ -9,8 +9,10 @@ compiler traces through the layer without a graph break (checked with
 torch._dynamo.explain).  Here:
 
 * ``torch.ops.lora_b200.lora_linear(X, W, A, B, scale)`` runs ``lora_fwd``;
-* ``torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, scale)`` runs
-  ``lora_bwd`` and returns (dX, dA, dB);
+* ``torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, scale, fp32_grads)``
+  runs ``lora_bwd_ex`` and returns (dX, dA, dB), dA and dB in fp32 when
+  ``fp32_grads`` (the unrounded reductions, e.g. for fp32 optimizer states
+  or a data-parallel sum before rounding), else bf16;
 * both have fake (meta) implementations, so they trace under FakeTensorMode
   and torch.compile without graph breaks, and the first is differentiable
   in X, A and B through the second.  W is frozen: it gets no gradient.
@@ -32,7 +34,7 @@ from typing import Optional, Tuple
 
 import torch
 
-from . import lora_bwd, lora_bwd_workspace_size, lora_fwd
+from . import LORA_BWD_FP32_GRADS, lora_bwd_ex, lora_bwd_workspace_size, lora_fwd
 
 _LIB = "lora_b200"
 
@@ -65,22 +67,25 @@ def _lora_linear_fake(X, W, A, B, scale):
 
 @torch.library.custom_op(f"{_LIB}::lora_linear_bwd", mutates_args=())
 def lora_linear_bwd(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, dY: torch.Tensor,
-                    scale: float) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """(dX, dA, dB) of Y = X W^T + scale (X A^T) B^T for the gradient dY."""
+                    scale: float, fp32_grads: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(dX, dA, dB) of Y = X W^T + scale (X A^T) B^T for the gradient dY;
+    dA and dB in fp32 when fp32_grads, else in the dtype of A and B."""
     M, d_in, d_out, r = _check(X, W, A, B)
+    gdt = torch.float32 if fp32_grads else A.dtype
     dX = torch.empty((M, d_in), dtype=X.dtype, device=X.device)
-    dA = torch.empty((r, d_in), dtype=A.dtype, device=A.device)
-    dB = torch.empty((d_out, r), dtype=B.dtype, device=B.device)
+    dA = torch.empty((r, d_in), dtype=gdt, device=A.device)
+    dB = torch.empty((d_out, r), dtype=gdt, device=B.device)
     ws = torch.empty(max(lora_bwd_workspace_size(M, d_in, d_out, r), 1), dtype=torch.uint8, device=X.device)
-    lora_bwd(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
-             scale * r, ws)
+    lora_bwd_ex(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
+                scale * r, ws, LORA_BWD_FP32_GRADS if fp32_grads else 0)
     return dX, dA, dB
 
 
 @lora_linear_bwd.register_fake
-def _lora_linear_bwd_fake(X, W, A, B, dY, scale):
+def _lora_linear_bwd_fake(X, W, A, B, dY, scale, fp32_grads=False):
     M, d_in, d_out, r = _check(X, W, A, B)
-    return X.new_empty((M, d_in)), A.new_empty((r, d_in)), B.new_empty((d_out, r))
+    gdt = torch.float32 if fp32_grads else A.dtype
+    return X.new_empty((M, d_in)), A.new_empty((r, d_in), dtype=gdt), B.new_empty((d_out, r), dtype=gdt)
 
 
 def _setup_context(ctx, inputs, output):

@@ -16,12 +16,12 @@ def test_library_loads_and_exports_every_header_function(built_lib):
     so = L.lib()
     for n in names:
         assert hasattr(so, n), f"{n} declared in include/lora.h but not exported"
-    assert L.lora_abi_version() == 1
+    assert L.lora_abi_version() == 2
 
 
 def test_header_declares_the_hot_path_entry_points(built_lib):
     names = set(built_lib.header_functions())
-    for n in ("lora_fwd", "lora_bwd", "lora_bwd_workspace_size", "lora_merge", "lora_merge_batched",
+    for n in ("lora_fwd", "lora_bwd", "lora_bwd_ex", "lora_bwd_workspace_size", "lora_merge", "lora_merge_batched",
               "lora_restore", "lora_get_device_status", "lora_check_args", "lora_status_string"):
         assert n in names
 
@@ -151,3 +151,19 @@ def test_fwd_batched_validation_before_any_cuda_call(built_lib):
     assert call([ok_a, (*b[:4], a[0] + 4096, 128, 1024, 256)]) == "LORA_ERR_ALIAS"
     # two entries share one Y
     assert call([ok_a, (*b[:4], a[4], 128, 1024, 256)]) == "LORA_ERR_ALIAS"
+
+
+def test_bwd_ex_refuses_unknown_flags_before_any_cuda_call(built_lib):
+    """The flags word is checked first: an unknown bit is LORA_ERR_FLAGS even
+    with pointers that are never dereferenced and no GPU present."""
+    L = built_lib
+    so = L.lib()
+    p = [ctypes.c_void_p(x) for x in _ptrs(9)]
+    args = p[:8] + [256, 512, 512, 16, ctypes.c_float(32.0), p[8], 1 << 30]
+    for flags in (2, 4, 0x80000000, 0xFFFFFFFE):
+        assert L.STATUS[so.lora_bwd_ex(*args, flags, None)] == "LORA_ERR_FLAGS"
+    # known flags pass validation and stop at the device check only on a GPU-less host
+    bad_align = list(p)
+    bad_align[6] = ctypes.c_void_p(ALIGNED + 8)        # dA not 16-byte aligned
+    code = so.lora_bwd_ex(*(bad_align[:8] + args[8:]), L.LORA_BWD_FP32_GRADS, None)
+    assert L.STATUS[code] == "LORA_ERR_ALIGN"

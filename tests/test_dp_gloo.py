@@ -4,7 +4,9 @@ Each rank takes its shard of the tokens, runs the fp64 oracle's backward on
 it, and the adapter gradients are summed with lora_linear_layer_b200.dp's
 all-reduce.  The summed dA, dB and the concatenated dX shards must equal the
 oracle on the whole batch, and the timing reduction must return the maximum
-over ranks.  No GPU is involved."""
+over ranks.  The partials are summed in fp64, and in fp32 as the GPU path
+does (lora_bwd_ex with fp32 gradients, summed before any rounding).  No GPU
+is involved."""
 import os
 import socket
 import sys
@@ -23,7 +25,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, M, q):
+def _worker(rank, world, port, M, q, dtype="float64"):
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
 
@@ -42,7 +44,8 @@ def _worker(rank, world, port, M, q):
         X, W, A, B, dY = (f(t[k]) for k in ("X", "W", "A", "B", "dY"))
         b, e = dp.shard_rows(M, world, rank)
         dX, dA, dB = O.lora_backward(X[b:e], W, A, B, dY[b:e], sh.alpha)
-        dA_t, dB_t = torch.from_numpy(dA.copy()), torch.from_numpy(dB.copy())
+        dA_t = torch.from_numpy(dA.astype(dtype))
+        dB_t = torch.from_numpy(dB.astype(dtype))
         dp.allreduce_adapter_grads(dA_t, dB_t)
         times = dp.max_over_ranks([1.0 + rank, 5.0 - rank])
         q.put((rank, b, e, dX, dA_t.numpy(), dB_t.numpy(), times))
@@ -50,8 +53,8 @@ def _worker(rank, world, port, M, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("M", [16, 23])
-def test_two_rank_backward_equals_full_batch(M):
+@pytest.mark.parametrize("M,dtype", [(16, "float64"), (23, "float64"), (23, "float32")])
+def test_two_rank_backward_equals_full_batch(M, dtype):
     sys.path.insert(0, ROOT)
     import oracle as O
     import workloads as WL
@@ -59,7 +62,7 @@ def test_two_rank_backward_equals_full_batch(M):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, M, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, M, q, dtype)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted([q.get(timeout=120) for _ in range(world)], key=lambda x: x[0])
@@ -73,9 +76,11 @@ def test_two_rank_backward_equals_full_batch(M):
     # shards cover the rows exactly once, in order
     assert [(r[1], r[2]) for r in res] == [(0, (M + 1) // 2), ((M + 1) // 2, M)]
     np.testing.assert_allclose(np.concatenate([r[3] for r in res]), dX, rtol=1e-12, atol=1e-12)
+    tol = 1e-12 if dtype == "float64" else 2e-6    # a few fp32 roundings
     for r in res:   # every rank holds the full-batch sums after the all-reduce
-        np.testing.assert_allclose(r[4], dA, rtol=1e-12, atol=1e-12)
-        np.testing.assert_allclose(r[5], dB, rtol=1e-12, atol=1e-12)
+        assert r[4].dtype == np.dtype(dtype) and r[5].dtype == np.dtype(dtype)
+        np.testing.assert_allclose(r[4], dA, rtol=tol, atol=tol * np.abs(dA).max())
+        np.testing.assert_allclose(r[5], dB, rtol=tol, atol=tol * np.abs(dB).max())
         assert r[6] == [2.0, 5.0]
 
 

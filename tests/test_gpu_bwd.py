@@ -103,3 +103,37 @@ def test_bwd_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in
     t = WL.make_layer_inputs(sh, seed=13, with_dy=True)
     dX, dA, dB = run_bwd(gpu, t["X"], t["W"], t["A"], t["B"], t["dY"], alpha)
     _check_all(t, alpha, dX, dA, dB)
+
+
+# (M, d_in, d_out, r): one split per row tile (no cluster reduction), the
+# in-cluster reduction with a ragged last split, r = 128, and an empty batch
+FP32_SHAPES = [(1, 8, 8, 8), (300, 520, 264, 8), (4100, 1024, 1536, 32), (257, 256, 384, 128), (0, 512, 264, 24)]
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r", FP32_SHAPES)
+def test_bwd_fp32_grads_round_to_the_bf16_results(gpu, M, d_in, d_out, r):
+    """lora_bwd_ex with LORA_BWD_FP32_GRADS: dA and dB are the fp32 sums
+    lora_bwd rounds, so rounding them (RNE) reproduces lora_bwd's bf16 dA and
+    dB bit for bit; dX is unchanged; the fp32 values meet the tolerance."""
+    alpha = 2.0 * r
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=17 + M, with_dy=True)
+    dX16, dA16, dB16 = run_bwd(gpu, t["X"], t["W"], t["A"], t["B"], t["dY"], alpha)
+    Xd, Wd, Ad, Bd, dYd = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    nan = float("nan")
+    dX = torch.full((M, d_in), nan, dtype=torch.bfloat16, device="cuda")
+    dA = torch.full((r, d_in), nan, dtype=torch.float32, device="cuda")
+    dB = torch.full((d_out, r), nan, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(gpu.lora_bwd_workspace_size(M, d_in, d_out, r), 256), dtype=torch.uint8, device="cuda")
+    gpu.lora_bwd_ex(Xd, Wd, Ad, Bd, dYd, dX, dA, dB, alpha, ws, gpu.LORA_BWD_FP32_GRADS)
+    assert gpu.lora_get_device_status() == 0
+    assert torch.equal(dX, dX16)
+    assert torch.equal(dA.to(torch.bfloat16), dA16) and torch.equal(dB.to(torch.bfloat16), dB16)
+    if M == 0:
+        assert not dA.any() and not dB.any()
+        return
+    ref_dX, ref_dA, ref_dB = O.lora_backward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]),
+                                             f64(t["dY"]), alpha)
+    for name, got, ref in (("dA", dA.double().cpu().numpy(), ref_dA), ("dB", dB.double().cpu().numpy(), ref_dB)):
+        ok, info = lora_tol_check(got, ref)
+        assert ok, (name, info)

@@ -83,3 +83,20 @@ def test_opcheck_schema_and_fake(gpu):
                           test_utils=("test_schema", "test_faketensor"))
     torch.library.opcheck(torch.ops.lora_b200.lora_linear_bwd.default, (X, W, A, B, dY, 0.75),
                           test_utils=("test_schema", "test_faketensor"))
+
+
+def test_backward_op_fp32_grads(gpu):
+    """lora_linear_bwd(..., fp32_grads=True): fp32 dA, dB that round to the
+    bf16 op's results bit for bit; dX identical."""
+    g = torch.Generator().manual_seed(41)
+    M, d_in, d_out, r = 384, 256, 320, 16
+    X = torch.randn(M, d_in, generator=g).to(torch.bfloat16).cuda()
+    W = (torch.randn(d_out, d_in, generator=g) * d_in ** -0.5).to(torch.bfloat16).cuda()
+    A = (torch.randn(r, d_in, generator=g) * d_in ** -0.5).to(torch.bfloat16).cuda()
+    B = (torch.randn(d_out, r, generator=g) * 0.02).to(torch.bfloat16).cuda()
+    dY = torch.randn(M, d_out, generator=g).to(torch.bfloat16).cuda()
+    dX16, dA16, dB16 = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, 0.75)
+    dX, dA, dB = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, 0.75, True)
+    assert dA.dtype == torch.float32 and dB.dtype == torch.float32
+    assert torch.equal(dX, dX16)
+    assert torch.equal(dA.to(torch.bfloat16), dA16) and torch.equal(dB.to(torch.bfloat16), dB16)

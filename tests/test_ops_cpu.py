@@ -86,3 +86,13 @@ def test_dynamo_traces_without_graph_breaks():
     ex = torch._dynamo.explain(f)(*args)
     assert ex.graph_break_count == 0
     assert ex.graph_count == 1
+
+
+def test_fake_backward_fp32_grads_dtype():
+    with FakeTensorMode():
+        X, W, A, B = _fake_inputs()
+        dY = torch.empty(32, 48, dtype=torch.bfloat16)
+        dX, dA, dB = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, 0.5, True)
+        assert dX.dtype == torch.bfloat16 and dA.dtype == torch.float32 and dB.dtype == torch.float32
+        dX, dA, dB = torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, 0.5)
+        assert dA.dtype == torch.bfloat16 and dB.dtype == torch.bfloat16
