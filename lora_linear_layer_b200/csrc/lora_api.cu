@@ -488,7 +488,11 @@ int splitk_mode() {
 // whose shortest contraction has `min_nk` K blocks: S CTAs (at most 8, the
 // portable cluster size) per tile, as many as fill the SMs, with at least 8
 // K blocks each (shorter K loops do not pay for the reduction: measured
-// slower at K = 512 and at 4 K blocks per split).
+// slower at K = 512 and at 4 K blocks per split).  From r_pad = 64 on, whose
+// T reduction costs more, contractions under 32 K blocks are not split: at
+// r = 64 two splits took 20.5 us on 128 x 1024 x 1024 and 512 x 1024 x 1024
+// against 16.4 us for one 128 x 128 tile per CTA (at K = 2048 four splits
+// and one tile per CTA tie, 20.5 us, and two splits take 22.6 us).
 // With more tiles than SMs (a grouped launch), three stages, so that two
 // CTAs fit on an SM.
 void plan_splitk(int64_t tiles, int min_nk, int r, int sm_count, SplitkPlan& pl) {
@@ -496,6 +500,7 @@ void plan_splitk(int64_t tiles, int min_nk, int r, int sm_count, SplitkPlan& pl)
   pl.RCW = rcw_of(pl.r_pad);
   pl.n_rchunks = (pl.r_pad + pl.RCW - 1) / pl.RCW;
   pl.splits = int(std::max<int64_t>(1, std::min<int64_t>({8, sm_count / std::max<int64_t>(1, tiles), min_nk / 8})));
+  if (pl.r_pad >= 64 && min_nk < 32) pl.splits = 1;
   int stages = tiles > sm_count ? 3 : 6;
   while (stages > 1 && SplitkLayout(pl.RCW, pl.r_pad, pl.n_rchunks, stages).total + 1024 > kSmemMax) --stages;
   pl.stages = stages;
