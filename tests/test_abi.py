@@ -167,3 +167,17 @@ def test_bwd_ex_refuses_unknown_flags_before_any_cuda_call(built_lib):
     bad_align[6] = ctypes.c_void_p(ALIGNED + 8)        # dA not 16-byte aligned
     code = so.lora_bwd_ex(*(bad_align[:8] + args[8:]), L.LORA_BWD_FP32_GRADS, None)
     assert L.STATUS[code] == "LORA_ERR_ALIGN"
+
+
+def test_size_limits(built_lib):
+    """Sizes up to 2^30 rows / columns pass validation, one step past is
+    LORA_ERR_SHAPE (validation only: the pointers are never dereferenced)."""
+    L = built_lib
+    big = 1 << 30
+    p = _ptrs(5, step=1 << 42)       # 4 TiB apart: a 2^30-row tensor is 1 TiB here
+    assert L.STATUS[L.lora_check_args(0, p, big, 512, 512, 16)] == "LORA_OK"
+    assert L.STATUS[L.lora_check_args(0, p, big + 1, 512, 512, 16)] == "LORA_ERR_SHAPE"
+    assert L.STATUS[L.lora_check_args(0, p, 256, big, 512, 16)] == "LORA_OK"
+    assert L.STATUS[L.lora_check_args(0, p, 256, big + 8, 512, 16)] == "LORA_ERR_SHAPE"
+    assert L.STATUS[L.lora_check_args(0, p, 256, 512, big + 8, 16)] == "LORA_ERR_SHAPE"
+    assert L.lora_bwd_workspace_size(big + 1, 512, 512, 16) == 0
