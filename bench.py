@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -79,11 +80,20 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text):
+    """C++ source with comments and blank space removed, so that the hash
+    below changes with the code, not with its comments (no '//' or '/*'
+    appears inside a string literal in these files)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
 def kernel_src_hash():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(_ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(_ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

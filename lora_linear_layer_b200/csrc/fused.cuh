@@ -23,15 +23,15 @@
 //   * four epilogue warps drain T, scale it by s in fp32, round to bf16 and
 //     write it into shared memory in the UMMA K-major swizzled layout (it
 //     never goes to global memory in the forward);
-//   * one more MMA pass (K = r) accumulates (sT) V^T onto the base
-//     accumulator; the epilogue rounds once to bf16 and writes OUT with
-//     TMA stores of 32 x 32 boxes staged in shared memory.
+//   * the tile's V rows arrive through the same ring, as one more stage
+//     after its K blocks; one more MMA pass (K = r) accumulates (sT) V^T
+//     onto the base accumulator; the epilogue rounds once to bf16 and
+//     writes OUT with TMA stores of 32 x 32 boxes staged in shared memory.
 // T is kept in shared memory and reused for every following tile of the
 // same M block (the schedule gives a cluster runs of consecutive N tiles of
 // one M block).  dX tiles have none of the T, U, V steps and take single-tile
-// runs.  Warp roles: warp 0 = TMA producer, warp 1 =
-// MMA issuer and TMEM owner, warps 2..5 = epilogue (warp w reads TMEM lanes
-// 32*(w%4)...).
+// runs.  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM
+// owner, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)...).
 //
 // CG = 2 runs each tile on a CTA pair (a cluster of two, cta_group::2):
 // each CTA holds its own 128 rows of P and half of the Q/U/V rows, the even
