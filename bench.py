@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # configuration / schedule)
 KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
                   "lora_linear_layer_b200/csrc/common.cuh", "lora_linear_layer_b200/csrc/lora_api.cu")
-LAUNCHES_PER_STEP = 5   # fwd 1; bwd: T + dT, dX, dB + dA; merge 1
+LAUNCHES_PER_STEP = 5   # fwd 1; bwd: T + dT, dB + dA, dX; merge 1
 
 
 # ------------------------------------------------------ algorithmic work ----

@@ -108,8 +108,9 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
  *   dA[r, d_in]  = dT^T X            (bf16, reduced over M in fp32)
  *   dB[d_out, r] = s dY^T T          (bf16, reduced over M in fp32)
  * with T = X A^T recomputed and dT = s dY B, both rounded to bf16 and kept
- * in the workspace by a first launch; dX is then one product over the
- * contraction [d_out | r], dY W + dT A, rounded once.
+ * in the workspace by a first launch; a second launch reduces dA and dB;
+ * dX is then one product over the contraction [d_out | r], dY W + dT A,
+ * rounded once.
  * `workspace` is caller-owned device memory of at least
  * lora_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on
  * entry do not matter and are clobbered.  Results are bitwise repeatable:

@@ -1032,22 +1032,7 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
                       : launch_skinny<false>(mp_t, mr_t, ct, st, &mp_dt, &mr_dt, &cdt);
     if (s != LORA_OK) return s;
   }
-  // 2. dX = dY W + dT A: one GEMM over the contraction [d_out | r_pad]
-  {
-    FusedCfg c;
-    if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
-    c.args.scale = 1.0f;
-    c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
-    CUtensorMap maps[5];
-    if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
-        !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
-        !make_map(&maps[2], dTws, r_pad, M, r_pad, 64, 128, 128) ||
-        !make_map(&maps[3], A, d_in, r, d_in, 64, 64, 128) ||
-        !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
-      return LORA_ERR_CUDA;
-    if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
-  }
-  // 3 + 4, one launch:  dB = s * sum_m dY[m, i] T[m, j]  and
+  // 2. One launch:  dB = s * sum_m dY[m, i] T[m, j]  and
   //                     dA^T[i, j] = sum_m X[m, i] dT[m, j], written transposed into dA
   {
     CUtensorMap mp_b, mr_b, mp_a, mr_a;
@@ -1064,6 +1049,21 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
     ca.args.out = reinterpret_cast<__nv_bfloat16*>(dA);
     ca.args.out_f32 = f32 ? 1 : 0;
     if ((s = launch_skinny<true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
+  }
+  // 3. dX = dY W + dT A: one GEMM over the contraction [d_out | r_pad]
+  {
+    FusedCfg c;
+    if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
+    c.args.scale = 1.0f;
+    c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
+    CUtensorMap maps[5];
+    if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
+        !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
+        !make_map(&maps[2], dTws, r_pad, M, r_pad, 64, 128, 128) ||
+        !make_map(&maps[3], A, d_in, r, d_in, 64, 64, 128) ||
+        !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
+      return LORA_ERR_CUDA;
+    if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
   }
   return LORA_OK;
 }
