@@ -294,8 +294,12 @@ def run_ours(args):
         if ev_f1 is not None:
             ev_f1.record(stream)
         if world > 1:
-            L.lora_bwd_ex(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, L.LORA_BWD_FP32_GRADS, stream)
-            dp.allreduce_adapter_grads(dA, dB)   # the data-parallel exchange (NCCL), fp32
+            # dA and dB first; their exchange (NCCL, fp32) overlaps the dX step
+            L.lora_bwd_grads(Xb, A, B, dYb, dA, dB, alpha, ws, L.LORA_BWD_FP32_GRADS, stream)
+            works = dp.allreduce_adapter_grads(dA, dB, async_op=True)
+            L.lora_bwd_dx(W, A, dYb, dX, ws, stream)
+            for w in works:
+                w.wait()
         else:
             L.lora_bwd(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, stream)
         L.lora_merge(W, A, B, Wm, alpha, stream)

@@ -143,6 +143,28 @@ lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const voi
                           void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
 
 /*
+ * The backward of lora_bwd_ex in two calls on one workspace, for callers
+ * that want dA and dB before dX is computed, e.g. to start summing them
+ * across data-parallel ranks while dX runs:
+ *   lora_bwd_grads: T and dT into the workspace, then dA and dB (flags as in
+ *                   lora_bwd_ex);
+ *   lora_bwd_dx:    dX = dY W + dT A from the dT that the preceding
+ *                   lora_bwd_grads call of the same shape left in
+ *                   `workspace`.
+ * Called in that order on one stream (or with the second ordered after the
+ * first), with the same M, d_in, d_out, r and workspace, and nothing
+ * writing the workspace in between, they give exactly lora_bwd_ex's results,
+ * bit for bit.  Argument rules as lora_bwd_ex for the tensors each call
+ * takes.
+ */
+lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
+                             int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                             void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
+lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX,
+                          int64_t M, int64_t d_in, int64_t d_out, int32_t r,
+                          const void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward without a workspace argument (the pages describe no such entry
  * point; it is a service of this library, not part of the method).
  *

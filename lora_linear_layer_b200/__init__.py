@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
         L.lora_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, vp]
         L.lora_bwd_ex.restype = ctypes.c_int
         L.lora_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, ctypes.c_uint32, vp]
+        L.lora_bwd_grads.restype = ctypes.c_int
+        L.lora_bwd_grads.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, ctypes.c_uint32, vp]
+        L.lora_bwd_dx.restype = ctypes.c_int
+        L.lora_bwd_dx.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, sz, vp]
         L.lora_bwd_noalloc.restype = ctypes.c_int
         L.lora_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
         L.lora_merge.restype = ctypes.c_int
@@ -232,6 +236,43 @@ def lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, flags: int 
                              M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, int(flags),
                              _stream(stream))
     _raise(code, "lora_bwd_ex")
+
+
+def _check_grads(dA, dB, r: int, d_in: int, d_out: int, flags: int):
+    torch = _tm()
+    gdt = torch.float32 if int(flags) & LORA_BWD_FP32_GRADS else torch.bfloat16
+    for t, n, s in ((dA, "dA", (r, d_in)), (dB, "dB", (d_out, r))):
+        if not isinstance(t, torch.Tensor) or t.dtype != gdt:
+            raise TypeError(f"{n} must be a {gdt} tensor with these flags")
+        if not t.is_cuda or not t.is_contiguous() or t.shape != s:
+            raise ValueError(f"{n} must be a contiguous CUDA tensor of shape {s}")
+
+
+def lora_bwd_grads(X, A, B, dY, dA, dB, alpha: float, workspace, flags: int = 0, stream=None) -> None:
+    """First half of the backward (see include/lora.h): T and dT into the
+    workspace, then dA and dB.  lora_bwd_dx with the same workspace gives dX."""
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (dY, "dY", (M, d_out))):
+        _check_tensor(t, n, s)
+    _check_grads(dA, dB, r, d_in, d_out, flags)
+    ws_bytes = int(workspace.numel() * workspace.element_size())
+    code = lib().lora_bwd_grads(_ptr(X), _ptr(A), _ptr(B), _ptr(dY), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
+                                float(alpha), _ptr(workspace), ws_bytes, int(flags), _stream(stream))
+    _raise(code, "lora_bwd_grads")
+
+
+def lora_bwd_dx(W, A, dY, dX, workspace, stream=None) -> None:
+    """Second half of the backward: dX = dY W + dT A from the dT that the
+    preceding lora_bwd_grads call of the same shape left in `workspace`."""
+    M, d_out = dY.shape
+    r, d_in = A.shape
+    for t, n, s in ((W, "W", (d_out, d_in)), (A, "A", (r, d_in)), (dY, "dY", (M, d_out)), (dX, "dX", (M, d_in))):
+        _check_tensor(t, n, s)
+    ws_bytes = int(workspace.numel() * workspace.element_size())
+    code = lib().lora_bwd_dx(_ptr(W), _ptr(A), _ptr(dY), _ptr(dX), M, d_in, d_out, r, _ptr(workspace), ws_bytes,
+                             _stream(stream))
+    _raise(code, "lora_bwd_dx")
 
 
 def lora_bwd_noalloc(X, W, A, B, dY, dX, dA, dB, alpha: float, stream=None) -> None:

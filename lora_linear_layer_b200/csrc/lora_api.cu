@@ -986,24 +986,11 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
   return p.total;
 }
 
-// The backward, with `need` bytes of workspace required; `flags` as in
-// lora_bwd_ex.
-static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
-                             void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
-                             void* workspace, size_t workspace_bytes, size_t need, uint32_t flags, void* stream) {
-  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
-  const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
-  const int gb = f32 ? 4 : 2;  // bytes per dA / dB element
-  const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
-  lora_status_t s = check_bwd_args(ptrs, 9, M, d_in, d_out, r, workspace_bytes, need, gb);
-  if (s != LORA_OK) return s;
-  DeviceInfo dev;
-  if ((s = device_info(dev)) != LORA_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M == 0) {
-    if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
-    return zero_bytes(dB, size_t(d_out) * r * gb, st);
-  }
+// Launches 1 and 2 of the backward: T and dT into the workspace, then dA and
+// dB.  Arguments already validated, M > 0.
+static lora_status_t launch_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA,
+                                      void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                                      void* workspace, bool f32, cudaStream_t st) {
   BwdPlan p;
   plan_bwd(M, d_in, d_out, r, p);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
@@ -1012,7 +999,7 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
   const float scale = alpha / float(r);
   const int r_pad = r_pad_of(r);
   const int rcw = rcw_of(r_pad);
-
+  lora_status_t s = LORA_OK;
 
   // 1. One launch, two jobs: dT = s dY B and T = X A^T (recomputed), each
   //    bf16 [M, r_pad] with zero columns past r.  The longer contraction's
@@ -1050,10 +1037,23 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
     ca.args.out_f32 = f32 ? 1 : 0;
     if ((s = launch_skinny<true>(mp_b, mr_b, cb, st, &mp_a, &mr_a, &ca)) != LORA_OK) return s;
   }
+  return LORA_OK;
+}
+
+// Launch 3 of the backward: dX from dY, W, A and the workspace's dT.
+// Arguments already validated, M > 0.
+static lora_status_t launch_bwd_dx(const void* W, const void* A, const void* dY, void* dX, int64_t M, int64_t d_in,
+                                   int64_t d_out, int32_t r, const void* workspace, int sm_count, cudaStream_t st) {
+  BwdPlan p;
+  plan_bwd(M, d_in, d_out, r, p);
+  const __nv_bfloat16* dTws =
+      reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const uint8_t*>(workspace) + p.off_dt);
+  const int r_pad = r_pad_of(r);
+  lora_status_t s = LORA_OK;
   // 3. dX = dY W + dT A: one GEMM over the contraction [d_out | r_pad]
   {
     FusedCfg c;
-    if (!pick_fused(M, d_in, d_out, r, true, dev.sm_count, c)) return LORA_ERR_RANK;
+    if (!pick_fused(M, d_in, d_out, r, true, sm_count, c)) return LORA_ERR_RANK;
     c.args.scale = 1.0f;
     c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
     CUtensorMap maps[5];
@@ -1063,9 +1063,31 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
         !make_map(&maps[3], A, d_in, r, d_in, 64, 64, 128) ||
         !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
       return LORA_ERR_CUDA;
-    if ((s = launch_fused<true>(maps, c, dev.sm_count, st)) != LORA_OK) return s;
+    if ((s = launch_fused<true>(maps, c, sm_count, st)) != LORA_OK) return s;
   }
   return LORA_OK;
+}
+
+// The backward, with `need` bytes of workspace required; `flags` as in
+// lora_bwd_ex.
+static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                             void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                             void* workspace, size_t workspace_bytes, size_t need, uint32_t flags, void* stream) {
+  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
+  const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
+  const int gb = f32 ? 4 : 2;  // bytes per dA / dB element
+  const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
+  lora_status_t s = check_bwd_args(ptrs, 9, M, d_in, d_out, r, workspace_bytes, need, gb);
+  if (s != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
+    return zero_bytes(dB, size_t(d_out) * r * gb, st);
+  }
+  if ((s = launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32, st)) != LORA_OK) return s;
+  return launch_bwd_dx(W, A, dY, dX, M, d_in, d_out, r, workspace, dev.sm_count, st);
 }
 
 lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
@@ -1073,6 +1095,87 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
                        void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
                  lora_bwd_workspace_size(M, d_in, d_out, r), 0u, stream);
+}
+
+// Pointer rules of the two-call backward: `required` buffers are non-null,
+// every non-null buffer is 16-byte aligned, no output overlaps an input or
+// another output.
+struct BufSpec {
+  const void* p;
+  uint64_t bytes;
+  bool required;
+};
+
+static lora_status_t check_bufs(const BufSpec* in, int n_in, const BufSpec* out, int n_out) {
+  for (int pass = 0; pass < 2; ++pass) {
+    const BufSpec* b = pass == 0 ? in : out;
+    const int n = pass == 0 ? n_in : n_out;
+    for (int i = 0; i < n; ++i) {
+      if (b[i].required && b[i].p == nullptr) return LORA_ERR_NULL;
+      if (b[i].p != nullptr && !aligned16(b[i].p)) return LORA_ERR_ALIGN;
+    }
+  }
+  for (int o = 0; o < n_out; ++o) {
+    if (out[o].p == nullptr) continue;
+    const Range ro = range_of(out[o].p, out[o].bytes);
+    for (int i = 0; i < n_in; ++i)
+      if (in[i].p != nullptr && overlaps(ro, range_of(in[i].p, in[i].bytes))) return LORA_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < n_out; ++o2)
+      if (out[o2].p != nullptr && overlaps(ro, range_of(out[o2].p, out[o2].bytes))) return LORA_ERR_ALIAS;
+  }
+  return LORA_OK;
+}
+
+// The workspace rule of lora_bwd for the two-call form.
+static lora_status_t check_workspace(const void* workspace, size_t workspace_bytes, size_t need) {
+  if (need == 0) return LORA_OK;
+  if (workspace == nullptr || workspace_bytes < need) return LORA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LORA_ERR_ALIGN;
+  return LORA_OK;
+}
+
+lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
+                             int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
+                             size_t workspace_bytes, uint32_t flags, void* stream) {
+  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
+  lora_status_t s = check_sizes(M, d_in, d_out, r);
+  if (s != LORA_OK) return s;
+  const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
+  const uint64_t gb = f32 ? 4 : 2;
+  const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != LORA_OK) return s;
+  const bool rows = M > 0;
+  const BufSpec in[4] = {{X, uint64_t(M) * d_in * 2, rows}, {A, uint64_t(r) * d_in * 2, true},
+                         {B, uint64_t(d_out) * r * 2, true}, {dY, uint64_t(M) * d_out * 2, rows}};
+  const BufSpec out[3] = {{dA, uint64_t(r) * d_in * gb, true}, {dB, uint64_t(d_out) * r * gb, true},
+                          {rows ? workspace : nullptr, need, rows}};
+  if ((s = check_bufs(in, 4, out, 3)) != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!rows) {
+    if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
+    return zero_bytes(dB, size_t(d_out) * r * gb, st);
+  }
+  return launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32, st);
+}
+
+lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX, int64_t M, int64_t d_in,
+                          int64_t d_out, int32_t r, const void* workspace, size_t workspace_bytes, void* stream) {
+  lora_status_t s = check_sizes(M, d_in, d_out, r);
+  if (s != LORA_OK) return s;
+  const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != LORA_OK) return s;
+  const bool rows = M > 0;
+  const BufSpec in[4] = {{W, uint64_t(d_out) * d_in * 2, true}, {A, uint64_t(r) * d_in * 2, true},
+                         {dY, uint64_t(M) * d_out * 2, rows}, {rows ? workspace : nullptr, need, rows}};
+  const BufSpec out[1] = {{dX, uint64_t(M) * d_in * 2, rows}};
+  if ((s = check_bufs(in, 4, out, 1)) != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  if (!rows) return LORA_OK;
+  return launch_bwd_dx(W, A, dY, dX, M, d_in, d_out, r, workspace, dev.sm_count,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,

@@ -26,12 +26,17 @@ def shard_rows(M: int, world: int, rank: int) -> Tuple[int, int]:
     return begin, begin + base + (1 if rank < extra else 0)
 
 
-def allreduce_adapter_grads(dA, dB, group=None) -> None:
+def allreduce_adapter_grads(dA, dB, group=None, async_op: bool = False):
     """Sum dA and dB over the ranks of `group`, in place (one all-reduce
-    each; the same collective order on every rank)."""
+    each; the same collective order on every rank).  With async_op the two
+    collectives are only enqueued (on NCCL they start once the work already
+    on the current stream is done) and their work handles are returned, so
+    that later kernels (the dX step) run while they are in flight; call
+    .wait() on each before dA and dB are read."""
     import torch.distributed as dist
-    dist.all_reduce(dA, op=dist.ReduceOp.SUM, group=group)
-    dist.all_reduce(dB, op=dist.ReduceOp.SUM, group=group)
+    w1 = dist.all_reduce(dA, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
+    w2 = dist.all_reduce(dB, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
+    return [w1, w2] if async_op else None
 
 
 def max_over_ranks(values, device=None, group=None):

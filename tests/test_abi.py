@@ -181,3 +181,31 @@ def test_size_limits(built_lib):
     assert L.STATUS[L.lora_check_args(0, p, 256, big + 8, 512, 16)] == "LORA_ERR_SHAPE"
     assert L.STATUS[L.lora_check_args(0, p, 256, 512, big + 8, 16)] == "LORA_ERR_SHAPE"
     assert L.lora_bwd_workspace_size(big + 1, 512, 512, 16) == 0
+
+
+def test_two_call_backward_validation(built_lib):
+    """lora_bwd_grads / lora_bwd_dx refuse bad arguments on the host before
+    any CUDA call (the pointers are never dereferenced)."""
+    L = built_lib
+    so = L.lib()
+    M, d_in, d_out, r = 256, 512, 512, 16
+    need = L.lora_bwd_workspace_size(M, d_in, d_out, r)
+    X, A, B, dY, dA, dB, W, dX = _ptrs(8)
+    ws = ALIGNED + (20 << 32)
+    c = lambda *a: L.STATUS[so.lora_bwd_grads(*[ctypes.c_void_p(x) if isinstance(x, int) and x > 1 << 20 else x
+                                                  for x in a])]
+    f = ctypes.c_float(32.0)
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 2, None) == "LORA_ERR_FLAGS"
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need - 256, 0, None) == "LORA_ERR_WORKSPACE"
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws + 16, need, 0, None) == "LORA_ERR_ALIGN"
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, 12, f, ws, need, 0, None) == "LORA_ERR_RANK"
+    assert c(X, A, B, dY, X + 16, dB, M, d_in, d_out, r, f, ws, need, 0, None) == "LORA_ERR_ALIAS"
+    assert c(X, A, B, dY, dA, dA, M, d_in, d_out, r, f, ws, need, 0, None) == "LORA_ERR_ALIAS"
+    assert c(0, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 0, None) == "LORA_ERR_NULL"
+    d = lambda *a: L.STATUS[so.lora_bwd_dx(*[ctypes.c_void_p(x) if isinstance(x, int) and x > 1 << 20 else x
+                                               for x in a])]
+    assert d(W, A, dY, dX, M, d_in, d_out, r, ws, 0, None) == "LORA_ERR_WORKSPACE"
+    assert d(W, A, dY, ws + 256, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_ALIAS"   # dX inside the workspace
+    assert d(W, A, dY, W, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_ALIAS"
+    assert d(W, A, dY, dX + 8, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_ALIGN"
+    assert d(0, A, dY, dX, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_NULL"

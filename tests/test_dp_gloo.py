@@ -25,7 +25,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, M, q, dtype="float64"):
+def _worker(rank, world, port, M, q, dtype="float64", async_op=False):
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
 
@@ -46,15 +46,18 @@ def _worker(rank, world, port, M, q, dtype="float64"):
         dX, dA, dB = O.lora_backward(X[b:e], W, A, B, dY[b:e], sh.alpha)
         dA_t = torch.from_numpy(dA.astype(dtype))
         dB_t = torch.from_numpy(dB.astype(dtype))
-        dp.allreduce_adapter_grads(dA_t, dB_t)
+        works = dp.allreduce_adapter_grads(dA_t, dB_t, async_op=async_op)
+        for w in works or []:
+            w.wait()
         times = dp.max_over_ranks([1.0 + rank, 5.0 - rank])
         q.put((rank, b, e, dX, dA_t.numpy(), dB_t.numpy(), times))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("M,dtype", [(16, "float64"), (23, "float64"), (23, "float32")])
-def test_two_rank_backward_equals_full_batch(M, dtype):
+@pytest.mark.parametrize("M,dtype,async_op", [(16, "float64", False), (23, "float64", False), (23, "float32", False),
+                                              (23, "float32", True)])
+def test_two_rank_backward_equals_full_batch(M, dtype, async_op):
     sys.path.insert(0, ROOT)
     import oracle as O
     import workloads as WL
@@ -62,7 +65,7 @@ def test_two_rank_backward_equals_full_batch(M, dtype):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, M, q, dtype)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, M, q, dtype, async_op)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted([q.get(timeout=120) for _ in range(world)], key=lambda x: x[0])

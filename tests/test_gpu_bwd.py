@@ -137,3 +137,34 @@ def test_bwd_fp32_grads_round_to_the_bf16_results(gpu, M, d_in, d_out, r):
     for name, got, ref in (("dA", dA.double().cpu().numpy(), ref_dA), ("dB", dB.double().cpu().numpy(), ref_dB)):
         ok, info = lora_tol_check(got, ref)
         assert ok, (name, info)
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r", [(300, 520, 264, 8), (4100, 1024, 1536, 32), (257, 256, 384, 128),
+                                            (0, 512, 264, 24)])
+@pytest.mark.parametrize("fp32", [False, True])
+def test_two_call_backward_equals_one_call(gpu, M, d_in, d_out, r, fp32):
+    """lora_bwd_grads then lora_bwd_dx on one workspace give lora_bwd_ex's
+    dX, dA and dB bit for bit."""
+    alpha = 2.0 * r
+    sh = WL.LayerShape(M, d_in, d_out, r, alpha)
+    t = WL.make_layer_inputs(sh, seed=31 + M, with_dy=True)
+    X, W, A, B, dY = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    gdt = torch.float32 if fp32 else torch.bfloat16
+    flags = gpu.LORA_BWD_FP32_GRADS if fp32 else 0
+    nan = float("nan")
+
+    def outs():
+        return (torch.full((M, d_in), nan, dtype=torch.bfloat16, device="cuda"),
+                torch.full((r, d_in), nan, dtype=gdt, device="cuda"),
+                torch.full((d_out, r), nan, dtype=gdt, device="cuda"))
+    ws = torch.full((max(gpu.lora_bwd_workspace_size(M, d_in, d_out, r), 256),), 255, dtype=torch.uint8,
+                    device="cuda")
+    dX1, dA1, dB1 = outs()
+    gpu.lora_bwd_ex(X, W, A, B, dY, dX1, dA1, dB1, alpha, ws, flags)
+    ws.fill_(255)
+    dX2, dA2, dB2 = outs()
+    gpu.lora_bwd_grads(X, A, B, dY, dA2, dB2, alpha, ws, flags)
+    gpu.lora_bwd_dx(W, A, dY, dX2, ws)
+    assert gpu.lora_get_device_status() == 0
+    assert torch.equal(dA1, dA2) and torch.equal(dB1, dB2)
+    assert torch.equal(dX1, dX2)
