@@ -199,3 +199,23 @@ def test_fwd_batched_more_problems_than_one_launch(gpu):
         ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
         ok, info = lora_tol_check(f64(Y.cpu()), ref)
         assert ok, info
+
+
+@pytest.mark.parametrize("r", [8, 64, 128])
+def test_fwd_batched_other_ranks(gpu, r):
+    """Grouped launches at the smallest rank, at r = 64 (short contractions
+    are not split there) and at r = 128 (base and T in one N = 256 MMA)."""
+    alpha = 2.0 * r
+    shapes = [(300, 520, 264), (128, 1024, 512), (64, 4096, 1024), (700, 2048, 136)]
+    items, hosts = [], []
+    for i, (M, d_in, d_out) in enumerate(shapes):
+        t = WL.make_layer_inputs(WL.LayerShape(M, d_in, d_out, r, alpha), seed=300 + 10 * r + i)
+        X, W, A, B = (dev(t[k]) for k in ("X", "W", "A", "B"))
+        items.append((X, W, A, B, torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device="cuda")))
+        hosts.append(t)
+    gpu.lora_fwd_batched(items, alpha)
+    assert gpu.lora_get_device_status() == 0
+    for (X, W, A, B, Y), t in zip(items, hosts):
+        ref = O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha)
+        ok, info = lora_tol_check(f64(Y.cpu()), ref)
+        assert ok, (r, tuple(X.shape), tuple(W.shape), info)
