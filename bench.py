@@ -285,24 +285,29 @@ def run_ours(args):
     ws = torch.empty(L.lora_bwd_workspace_size(M, d_in, d_out, r), dtype=torch.uint8, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    # --saved-t: the forward keeps T for the backward (one pass over X less)
+    bwd_flags = L.LORA_BWD_T_SAVED if args.saved_t else 0
 
     def step(ev_f0=None, ev_f1=None, Xb=None, dYb=None):
         Xb = X if Xb is None else Xb
         dYb = dY if dYb is None else dYb
         if ev_f0 is not None:
             ev_f0.record(stream)
-        L.lora_fwd(Xb, W, A, B, Y, alpha, stream)
+        if args.saved_t:
+            L.lora_fwd_save(Xb, W, A, B, Y, alpha, ws, stream)     # Y, and T into the workspace
+        else:
+            L.lora_fwd(Xb, W, A, B, Y, alpha, stream)
         if ev_f1 is not None:
             ev_f1.record(stream)
         if world > 1:
             # dA and dB first; their exchange (NCCL, fp32) overlaps the dX step
-            L.lora_bwd_grads(Xb, A, B, dYb, dA, dB, alpha, ws, L.LORA_BWD_FP32_GRADS, stream)
+            L.lora_bwd_grads(Xb, A, B, dYb, dA, dB, alpha, ws, L.LORA_BWD_FP32_GRADS | bwd_flags, stream)
             works = dp.allreduce_adapter_grads(dA, dB, async_op=True)
             L.lora_bwd_dx(W, A, dYb, dX, ws, stream)
             for w in works:
                 w.wait()
         else:
-            L.lora_bwd(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, stream)
+            L.lora_bwd_ex(Xb, W, A, B, dYb, dX, dA, dB, alpha, ws, bwd_flags, stream)
         L.lora_merge(W, A, B, Wm, alpha, stream)
 
     warm = max(3, args.warmup)
@@ -420,7 +425,8 @@ def run_ours(args):
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded normal inputs, bf16)",
         "config": {"workload": sh.name, "M": M, "d_in": d_in, "d_out": d_out, "r": r, "alpha": alpha,
-                   "global_batch_tokens": M * world, "step": "lora_fwd + lora_bwd + lora_merge",
+                   "global_batch_tokens": M * world, "step": ("lora_fwd_save + lora_bwd_ex (T saved) + lora_merge" if args.saved_t
+                            else "lora_fwd + lora_bwd + lora_merge"),
                    "l2": "flushed between steps (256 MB write outside the timed pairs); inputs > L2",
                    "parallelism": f"dp{world}" if world > 1 else "single GPU"},
         "breakdown": {"fwd_us": 1e3 * fwd_avg_ms, "fwd_tflops": achieved,
@@ -550,7 +556,10 @@ def compare_shapes():
 def run_compare(args):
     """Unfused PyTorch LoRA (cuBLAS matmuls, the pages' six-launch forward and
     its autograd backward with W frozen) against lora_fwd / lora_bwd: median
-    device time of each, L2 flushed before every call, and the speedup."""
+    device time of each, L2 flushed before every call, and the speedup.  The
+    unfused backward reuses the X A^T its forward kept; the same holds for
+    lora_bwd_ex with LORA_BWD_T_SAVED after lora_fwd_save, reported beside
+    lora_bwd (which recomputes T)."""
     import torch
     import lora_linear_layer_b200 as L
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -582,10 +591,14 @@ def run_compare(args):
         # forward alone and subtract it
         tfb = _time_events(torch_bwd, flush, n)[0]
         ob = _time_events(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n)[0]
+        L.lora_fwd_save(X, W, A, B, Y, sh.alpha, ws)       # T into the workspace, kept by the backward
+        obs = _time_events(lambda: L.lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws, L.LORA_BWD_T_SAVED),
+                           flush, n)[0]
         tb = max(tfb - _time_events(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n)[0], 1e-3)
         print(json.dumps({"point": sh.name, "M": sh.M, "d_in": sh.d_in, "d_out": sh.d_out, "r": sh.r,
                           "torch_fwd_us": tf, "ours_fwd_us": of, "fwd_speedup": tf / of,
                           "torch_bwd_us": tb, "ours_bwd_us": ob, "bwd_speedup": tb / ob,
+                          "ours_bwd_saved_t_us": obs, "bwd_saved_t_speedup": tb / obs,
                           "torch": "unfused: X@W.T + (X@A.T)@B.T*s, autograd backward (W frozen)",
                           "l2": "flushed before every call"}), flush=True)
         del X, W, A, B, dY, Y, dX, dA, dB, ws, Xg, Ag, Bg
@@ -676,6 +689,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true", help="time lora_fwd on every sweep point (one line each)")
     ap.add_argument("--sweep-filter", default="", help="only sweep points whose name contains this")
+    ap.add_argument("--saved-t", action="store_true",
+                    help="the step keeps T from the forward: lora_fwd_save + lora_bwd_ex with LORA_BWD_T_SAVED")
     ap.add_argument("--merge", action="store_true", help="time the 252-matrix batched merge refresh")
     ap.add_argument("--tiny", action="store_true", help="time the tiny forward (eager and CUDA-graph replay)")
     ap.add_argument("--grouped", action="store_true",

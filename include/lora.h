@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define LORA_ABI_VERSION 2
+#define LORA_ABI_VERSION 3
 
 typedef enum {
   LORA_OK = 0,
@@ -96,6 +96,24 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
                        void* stream);
 
 /*
+ * Forward that also keeps T for the backward: Y exactly as lora_fwd (bit for
+ * bit), and T = X A^T (unscaled, each value the fp32 sum that the forward's
+ * up-projection scales, rounded once to bf16; zero columns past r) written
+ * into `workspace`, a buffer of at least lora_bwd_workspace_size(M, d_in,
+ * d_out, r) bytes, 256-byte aligned, that overlaps none of X, W, A, B, Y.
+ * Pass the same workspace to lora_bwd_ex or lora_bwd_grads with
+ * LORA_BWD_T_SAVED, which then skip recomputing T.  The T slot's layout is
+ * the library's own; only the workspace as a whole is passed along.
+ * In the tiled forward the tile of N index 0 of every M block stores its
+ * rows of T from the epilogue (no extra pass over X); in the split-contraction
+ * form for small outputs, T is one more launch that reads X.
+ * With M == 0 nothing happens (the workspace may then be NULL).
+ */
+lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const void* B, void* Y,
+                            int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device scratch lora_bwd needs for this shape (0 when M == 0).
  * Holds T and dT as bf16 [M, r_pad] (r_pad = r rounded up to 16), each at a
  * 256-byte aligned offset.
@@ -123,8 +141,9 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
                        int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                        void* workspace, size_t workspace_bytes, void* stream);
 
-/* Flags of lora_bwd_ex. */
+/* Flags of lora_bwd_ex and lora_bwd_grads. */
 #define LORA_BWD_FP32_GRADS 1u /* dA and dB are fp32 (float) instead of bf16 */
+#define LORA_BWD_T_SAVED 2u    /* the workspace already holds T from lora_fwd_save */
 
 /*
  * lora_bwd with flags.  flags == 0 is exactly lora_bwd.  With
@@ -134,8 +153,16 @@ lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* 
  * lora_bwd rounds to bf16 (RNE), so rounding them gives lora_bwd's results
  * bit for bit.  Meant for fp32 optimizer states and for summing per-rank
  * partial gradients in fp32 before a single rounding (data parallelism).
- * With M == 0 they are set to zero.  Other rules as lora_bwd; an unknown
- * flag bit returns LORA_ERR_FLAGS before anything is launched.
+ * With M == 0 they are set to zero.
+ * With LORA_BWD_T_SAVED the workspace must hold what a lora_fwd_save call
+ * of the same X, A and shape left there (nothing may have written the
+ * workspace since): T is not recomputed and the first launch reads dY alone
+ * (for dT), one pass over X less.  dB then uses the forward's T, rounded
+ * from the forward's own accumulation order, and dT is reduced with its own
+ * split of the contraction, so the results agree with those of flags == 0
+ * to within bf16 rounding of T and dT, not bit for bit.
+ * Other rules as lora_bwd; an unknown flag bit returns LORA_ERR_FLAGS
+ * before anything is launched.
  */
 lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const void* B,
                           const void* dY, void* dX, void* dA, void* dB,
@@ -146,8 +173,8 @@ lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const voi
  * The backward of lora_bwd_ex in two calls on one workspace, for callers
  * that want dA and dB before dX is computed, e.g. to start summing them
  * across data-parallel ranks while dX runs:
- *   lora_bwd_grads: T and dT into the workspace, then dA and dB (flags as in
- *                   lora_bwd_ex);
+ *   lora_bwd_grads: T (unless LORA_BWD_T_SAVED) and dT into the workspace,
+ *                   then dA and dB (flags as in lora_bwd_ex);
  *   lora_bwd_dx:    dX = dY W + dT A from the dT that the preceding
  *                   lora_bwd_grads call of the same shape left in
  *                   `workspace`.

@@ -24,6 +24,7 @@ STATUS = {
     7: "LORA_ERR_TIMEOUT", 8: "LORA_ERR_UNSUPPORTED_DEVICE", 9: "LORA_ERR_ALIAS", 10: "LORA_ERR_FLAGS",
 }
 LORA_BWD_FP32_GRADS = 1
+LORA_BWD_T_SAVED = 2
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 
@@ -70,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.lora_status_string.argtypes = [ctypes.c_int]
         L.lora_fwd.restype = ctypes.c_int
         L.lora_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp]
+        L.lora_fwd_save.restype = ctypes.c_int
+        L.lora_fwd_save.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, f32, vp, sz, vp]
         L.lora_fwd_batched.restype = ctypes.c_int
         L.lora_fwd_batched.argtypes = [ctypes.POINTER(_FwdDesc), i32, i32, f32, vp]
         L.lora_bwd_workspace_size.restype = sz
@@ -173,6 +176,21 @@ def lora_fwd(X, W, A, B, Y, alpha: float, stream=None) -> None:
     _raise(code, "lora_fwd")
 
 
+def lora_fwd_save(X, W, A, B, Y, alpha: float, workspace, stream=None) -> None:
+    """lora_fwd that also writes T = X A^T into the backward's workspace
+    (see include/lora.h); pass that workspace to lora_bwd_ex or
+    lora_bwd_grads with LORA_BWD_T_SAVED."""
+    M, d_in = X.shape
+    d_out, r = B.shape
+    for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
+        _check_tensor(t, n, s)
+    ws_bytes = int(workspace.numel() * workspace.element_size())
+    code = lib().lora_fwd_save(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r, float(alpha),
+                               _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(code, "lora_fwd_save")
+
+
 def lora_fwd_batched(items: Sequence[Tuple], alpha: float, stream=None) -> None:
     """One launch for several independent forwards (X, W, A, B, Y) that share
     the rank r and alpha (see include/lora.h)."""
@@ -249,8 +267,9 @@ def _check_grads(dA, dB, r: int, d_in: int, d_out: int, flags: int):
 
 
 def lora_bwd_grads(X, A, B, dY, dA, dB, alpha: float, workspace, flags: int = 0, stream=None) -> None:
-    """First half of the backward (see include/lora.h): T and dT into the
-    workspace, then dA and dB.  lora_bwd_dx with the same workspace gives dX."""
+    """First half of the backward (see include/lora.h): T (unless
+    LORA_BWD_T_SAVED) and dT into the workspace, then dA and dB.  lora_bwd_dx
+    with the same workspace gives dX."""
     M, d_in = X.shape
     d_out, r = B.shape
     for t, n, s in ((X, "X", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (dY, "dY", (M, d_out))):

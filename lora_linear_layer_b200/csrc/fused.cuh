@@ -21,8 +21,11 @@
 //     tcgen05.mma for the base product into a TMEM accumulator and, on that
 //     first tile, the N = r product T = P U^T into a second TMEM region;
 //   * four epilogue warps drain T, scale it by s in fp32, round to bf16 and
-//     write it into shared memory in the UMMA K-major swizzled layout (it
-//     never goes to global memory in the forward);
+//     write it into shared memory in the UMMA K-major swizzled layout; when
+//     the caller asks for T (t_out), the tile of N index 0 of each M block
+//     also writes the unscaled T, rounded to bf16, to global memory for the
+//     backward (every M block's tile 0 is the first tile of a run, so T is
+//     in the epilogue's registers there);
 //   * the tile's V rows arrive through the same ring, as one more stage
 //     after its K blocks; one more MMA pass (K = r) accumulates (sT) V^T
 //     onto the base accumulator; the epilogue rounds once to bf16 and
@@ -62,6 +65,7 @@ struct FusedArgs {
   int32_t ep_bufs;          // output staging buffers per epilogue warp (1 or 2)
   float scale;              // s = alpha / r (forward)
   __nv_bfloat16* out;       // [M, N] row-major, ld = N
+  __nv_bfloat16* t_out;     // forward: NULL, or T = P U^T as bf16 [M, r_pad], ld = r_pad
   int32_t num_m, num_n;     // tile counts (M tiles of 128 * CG rows)
   int32_t band_w, n_bands;  // column bands of the schedule
   int32_t run_l;            // 0: contiguous ranges; L > 0: runs of L N-tiles dealt round-robin
@@ -469,10 +473,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         ++ntt;
         tc_fence_after();
         const uint32_t t_col = kFold ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
+        const int t_row = m * (kBM * CG) + int(rank) * kBM + row;
+        __nv_bfloat16* const t_dst =
+            a.t_out != nullptr && n == 0 && t_row < a.M ? a.t_out + size_t(t_row) * size_t(a.r_pad) : nullptr;
         for (int col = 0; col < a.r_pad; col += 16) {
           uint32_t v[16];
           tmem_ld_x16(tmem + lane_base + t_col + uint32_t(col), v);
           tmem_ld_wait();
+          if (t_dst != nullptr) {
+            uint32_t tu[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tu[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* d = reinterpret_cast<uint4*>(t_dst + col);
+            d[0] = make_uint4(tu[0], tu[1], tu[2], tu[3]);
+            d[1] = make_uint4(tu[4], tu[5], tu[6], tu[7]);
+          }
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)

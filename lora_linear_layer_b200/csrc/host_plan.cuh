@@ -120,6 +120,7 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   a.n_rchunks = c.n_rchunks;
   a.stages = c.stages;
   a.ep_bufs = c.ep_bufs;
+  a.t_out = nullptr;
   a.num_m = num_m;
   a.num_n = num_n;
   // Column bands keep the operands the whole GPU touches at once well
@@ -421,6 +422,7 @@ lora_status_t launch_skinny(const CUtensorMap& p0, const CUtensorMap& r0, const 
 
 struct BwdPlan {
   SkinnyCfg dt_cfg, t_cfg, db_cfg, da_cfg;
+  SkinnyCfg dto_cfg;  // dT alone, when the forward saved T
   size_t off_t, off_dt, total;
 };
 
@@ -436,6 +438,7 @@ void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
   const int s1 = d_out >= d_in ? p.dt_cfg.splits : p.t_cfg.splits;
   resplit_skinny(p.dt_cfg, s1);
   resplit_skinny(p.t_cfg, s1);
+  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, (M + 127) / 128, p.dto_cfg);
   // dB and dA share one launch, so they share its split count
   const int64_t dbda_tiles = (d_out + 127) / 128 + (d_in + 127) / 128;
   pick_skinny(d_out, M, r, true, OUT_ROWS_R, dbda_tiles, p.db_cfg);

@@ -137,29 +137,44 @@ static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int
   }
 }
 
-lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
-                       int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
-  const void* ptrs[5] = {X, W, A, B, Y};
-  lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
-  if (s != LORA_OK) return s;
-  DeviceInfo dev;
-  if ((s = device_info(dev)) != LORA_OK) return s;
-  if (M == 0) return LORA_OK;
+// T = X A^T as bf16 [M, r_pad] (zero columns past r) into `Tws`: one
+// skinny launch.  Arguments already validated, M > 0.
+static lora_status_t launch_t(const void* X, const void* A, int64_t M, int64_t d_in, int32_t r,
+                              __nv_bfloat16* Tws, cudaStream_t st) {
+  SkinnyCfg ct;
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, (M + 127) / 128, ct);
+  ct.args.out = Tws;
+  CUtensorMap mp, mr;
+  if (!make_map(&mp, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr, A, d_in, r, d_in, 64, ct.r_pad, 128))
+    return LORA_ERR_CUDA;
+  return launch_skinny<false>(mp, mr, ct, st);
+}
+
+// The forward; when `Tws` is not NULL it also receives T = X A^T (bf16
+// [M, r_pad], zero columns past r).  Arguments already validated, M > 0.
+static lora_status_t fwd_run(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                             int64_t d_in, int64_t d_out, int32_t r, float alpha, __nv_bfloat16* Tws,
+                             int sm_count, cudaStream_t st) {
   {
     SplitkPlan pl;
-    if (use_splitk(M, d_out, d_in, r, dev.sm_count, pl)) {
+    if (use_splitk(M, d_out, d_in, r, sm_count, pl)) {
+      // split-K tiles each form their own partial T; the saved T is one
+      // more (skinny) launch
       SplitkTable<1> t;
       std::memset(&t, 0, sizeof(t));
       splitk_table_common(t, 1, pl, alpha / float(r));
       if (!splitk_job(t.job[0], X, W, A, B, Y, M, d_in, d_out, r, pl, 0)) return LORA_ERR_CUDA;
       const int tiles = int(((M + 127) / 128) * ((d_out + 127) / 128));
-      return launch_splitk(t, tiles, pl, reinterpret_cast<cudaStream_t>(stream));
+      const lora_status_t s = launch_splitk(t, tiles, pl, st);
+      if (s != LORA_OK || Tws == nullptr) return s;
+      return launch_t(X, A, M, d_in, r, Tws, st);
     }
   }
   FusedCfg c;
-  if (!pick_fused(M, d_out, d_in, r, false, dev.sm_count, c)) return LORA_ERR_RANK;
+  if (!pick_fused(M, d_out, d_in, r, false, sm_count, c)) return LORA_ERR_RANK;
   c.args.scale = alpha / float(r);
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
+  c.args.t_out = Tws;
   CUtensorMap maps[5];
   const uint32_t bnc = uint32_t(c.BN / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
@@ -168,7 +183,19 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
       !make_map(&maps[3], B, r, d_out, r, c.RCW, bnc, c.RCW * 2) ||
       !make_map(&maps[4], Y, d_out, M, d_out, kEpCols, 32, kEpCols * 2))
     return LORA_ERR_CUDA;
-  return launch_fused<false>(maps, c, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+  return launch_fused<false>(maps, c, sm_count, st);
+}
+
+lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                       int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
+  const void* ptrs[5] = {X, W, A, B, Y};
+  lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
+  if (s != LORA_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  if (M == 0) return LORA_OK;
+  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, alpha, nullptr, dev.sm_count,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
@@ -259,11 +286,12 @@ size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r
   return p.total;
 }
 
-// Launches 1 and 2 of the backward: T and dT into the workspace, then dA and
-// dB.  Arguments already validated, M > 0.
+// Launches 1 and 2 of the backward: T (unless `t_saved`: the forward left
+// it in the workspace) and dT into the workspace, then dA and dB.
+// Arguments already validated, M > 0.
 static lora_status_t launch_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA,
                                       void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
-                                      void* workspace, bool f32, cudaStream_t st) {
+                                      void* workspace, bool f32, bool t_saved, cudaStream_t st) {
   BwdPlan p;
   plan_bwd(M, d_in, d_out, r, p);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
@@ -277,7 +305,16 @@ static lora_status_t launch_bwd_grads(const void* X, const void* A, const void* 
   // 1. One launch, two jobs: dT = s dY B and T = X A^T (recomputed), each
   //    bf16 [M, r_pad] with zero columns past r.  The longer contraction's
   //    job takes the first row tiles of the grid, so it starts first.
-  {
+  //    With T saved by the forward: dT alone.
+  if (t_saved) {
+    CUtensorMap mp_dt, mr_dt;
+    if (!make_map(&mp_dt, dY, d_out, M, d_out, 64, 128, 128) || !make_map(&mr_dt, B, r, d_out, r, rcw, 64, rcw * 2))
+      return LORA_ERR_CUDA;
+    SkinnyCfg cdt = p.dto_cfg;
+    cdt.args.out = dTws;
+    cdt.args.scale = scale;
+    if ((s = launch_skinny<false>(mp_dt, mr_dt, cdt, st)) != LORA_OK) return s;
+  } else {
     CUtensorMap mp_dt, mr_dt, mp_t, mr_t;
     if (!make_map(&mp_dt, dY, d_out, M, d_out, 64, 128, 128) ||
         !make_map(&mr_dt, B, r, d_out, r, rcw, 64, rcw * 2) ||
@@ -346,7 +383,7 @@ static lora_status_t launch_bwd_dx(const void* W, const void* A, const void* dY,
 static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
                              void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                              void* workspace, size_t workspace_bytes, size_t need, uint32_t flags, void* stream) {
-  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
+  if ((flags & ~kBwdFlags) != 0u) return LORA_ERR_FLAGS;
   const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
   const int gb = f32 ? 4 : 2;  // bytes per dA / dB element
   const void* ptrs[9] = {X, W, A, B, dY, dX, dA, dB, workspace};
@@ -359,7 +396,9 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
     if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
     return zero_bytes(dB, size_t(d_out) * r * gb, st);
   }
-  if ((s = launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32, st)) != LORA_OK) return s;
+  if ((s = launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32,
+                            (flags & LORA_BWD_T_SAVED) != 0u, st)) != LORA_OK)
+    return s;
   return launch_bwd_dx(W, A, dY, dX, M, d_in, d_out, r, workspace, dev.sm_count, st);
 }
 
@@ -407,10 +446,34 @@ static lora_status_t check_workspace(const void* workspace, size_t workspace_byt
   return LORA_OK;
 }
 
+lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                            int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  const void* ptrs[5] = {X, W, A, B, Y};
+  lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
+  if (s != LORA_OK) return s;
+  const size_t need = lora_bwd_workspace_size(M, d_in, d_out, r);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != LORA_OK) return s;
+  if (M > 0) {
+    const Range ws = range_of(workspace, need);
+    const uint64_t bytes[5] = {uint64_t(M) * d_in * 2, uint64_t(d_out) * d_in * 2, uint64_t(r) * d_in * 2,
+                               uint64_t(d_out) * r * 2, uint64_t(M) * d_out * 2};
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(ws, range_of(ptrs[i], bytes[i]))) return LORA_ERR_ALIAS;
+  }
+  DeviceInfo dev;
+  if ((s = device_info(dev)) != LORA_OK) return s;
+  if (M == 0) return LORA_OK;
+  BwdPlan p;
+  plan_bwd(M, d_in, d_out, r, p);
+  __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(workspace) + p.off_t);
+  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, alpha, Tws, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
 lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
                              int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
                              size_t workspace_bytes, uint32_t flags, void* stream) {
-  if ((flags & ~LORA_BWD_FP32_GRADS) != 0u) return LORA_ERR_FLAGS;
+  if ((flags & ~kBwdFlags) != 0u) return LORA_ERR_FLAGS;
   lora_status_t s = check_sizes(M, d_in, d_out, r);
   if (s != LORA_OK) return s;
   const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
@@ -430,7 +493,8 @@ lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const 
     if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
     return zero_bytes(dB, size_t(d_out) * r * gb, st);
   }
-  return launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32, st);
+  return launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32,
+                          (flags & LORA_BWD_T_SAVED) != 0u, st);
 }
 
 lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX, int64_t M, int64_t d_in,

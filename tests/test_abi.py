@@ -16,12 +16,12 @@ def test_library_loads_and_exports_every_header_function(built_lib):
     so = L.lib()
     for n in names:
         assert hasattr(so, n), f"{n} declared in include/lora.h but not exported"
-    assert L.lora_abi_version() == 2
+    assert L.lora_abi_version() == 3
 
 
 def test_header_declares_the_hot_path_entry_points(built_lib):
     names = set(built_lib.header_functions())
-    for n in ("lora_fwd", "lora_bwd", "lora_bwd_ex", "lora_bwd_workspace_size", "lora_merge", "lora_merge_batched",
+    for n in ("lora_fwd", "lora_fwd_save", "lora_bwd", "lora_bwd_ex", "lora_bwd_workspace_size", "lora_merge", "lora_merge_batched",
               "lora_restore", "lora_get_device_status", "lora_check_args", "lora_status_string"):
         assert n in names
 
@@ -160,13 +160,14 @@ def test_bwd_ex_refuses_unknown_flags_before_any_cuda_call(built_lib):
     so = L.lib()
     p = [ctypes.c_void_p(x) for x in _ptrs(9)]
     args = p[:8] + [256, 512, 512, 16, ctypes.c_float(32.0), p[8], 1 << 30]
-    for flags in (2, 4, 0x80000000, 0xFFFFFFFE):
+    for flags in (4, 8, 0x80000000, 0xFFFFFFFC, 0xFFFFFFFF):
         assert L.STATUS[so.lora_bwd_ex(*args, flags, None)] == "LORA_ERR_FLAGS"
-    # known flags pass validation and stop at the device check only on a GPU-less host
+    # known flags pass the flags check and stop at the next rule (alignment)
     bad_align = list(p)
     bad_align[6] = ctypes.c_void_p(ALIGNED + 8)        # dA not 16-byte aligned
-    code = so.lora_bwd_ex(*(bad_align[:8] + args[8:]), L.LORA_BWD_FP32_GRADS, None)
-    assert L.STATUS[code] == "LORA_ERR_ALIGN"
+    for flags in (L.LORA_BWD_FP32_GRADS, L.LORA_BWD_T_SAVED, L.LORA_BWD_FP32_GRADS | L.LORA_BWD_T_SAVED):
+        code = so.lora_bwd_ex(*(bad_align[:8] + args[8:]), flags, None)
+        assert L.STATUS[code] == "LORA_ERR_ALIGN"
 
 
 def test_size_limits(built_lib):
@@ -195,7 +196,9 @@ def test_two_call_backward_validation(built_lib):
     c = lambda *a: L.STATUS[so.lora_bwd_grads(*[ctypes.c_void_p(x) if isinstance(x, int) and x > 1 << 20 else x
                                                   for x in a])]
     f = ctypes.c_float(32.0)
-    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 2, None) == "LORA_ERR_FLAGS"
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 4, None) == "LORA_ERR_FLAGS"
+    assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need - 256, L.LORA_BWD_T_SAVED,
+             None) == "LORA_ERR_WORKSPACE"
     assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need - 256, 0, None) == "LORA_ERR_WORKSPACE"
     assert c(X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws + 16, need, 0, None) == "LORA_ERR_ALIGN"
     assert c(X, A, B, dY, dA, dB, M, d_in, d_out, 12, f, ws, need, 0, None) == "LORA_ERR_RANK"
@@ -209,3 +212,27 @@ def test_two_call_backward_validation(built_lib):
     assert d(W, A, dY, W, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_ALIAS"
     assert d(W, A, dY, dX + 8, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_ALIGN"
     assert d(0, A, dY, dX, M, d_in, d_out, r, ws, need, None) == "LORA_ERR_NULL"
+
+
+def test_fwd_save_validation(built_lib):
+    """lora_fwd_save applies lora_fwd's rules plus the workspace rules of the
+    backward, and refuses a workspace that overlaps an input or Y, all on the
+    host before any CUDA call (the pointers are never dereferenced)."""
+    L = built_lib
+    so = L.lib()
+    M, d_in, d_out, r = 256, 512, 512, 16
+    need = L.lora_bwd_workspace_size(M, d_in, d_out, r)
+    X, W, A, B, Y = _ptrs(5)
+    ws = ALIGNED + (20 << 32)
+    c = lambda *a: L.STATUS[so.lora_fwd_save(*[ctypes.c_void_p(x) if isinstance(x, int) and x > 1 << 20 else x
+                                                 for x in a])]
+    f = ctypes.c_float(32.0)
+    assert c(X, W, A, B, Y, M, d_in, d_out, r, f, None, need, None) == "LORA_ERR_WORKSPACE"
+    assert c(X, W, A, B, Y, M, d_in, d_out, r, f, ws, need - 1, None) == "LORA_ERR_WORKSPACE"
+    assert c(X, W, A, B, Y, M, d_in, d_out, r, f, ws + 16, need, None) == "LORA_ERR_ALIGN"
+    for p in (X, W, A, B, Y):                    # the workspace starts inside each operand in turn
+        assert c(X, W, A, B, Y, M, d_in, d_out, r, f, p, need, None) == "LORA_ERR_ALIAS"
+    # lora_fwd's own rules come first
+    assert c(X, W, A, B, 0, M, d_in, d_out, r, f, ws, need, None) == "LORA_ERR_NULL"
+    assert c(X, W, A, B, Y, M, d_in, d_out, 12, f, ws, need, None) == "LORA_ERR_RANK"
+    assert c(X, W, A, B, X, M, d_in, d_out, r, f, ws, need, None) == "LORA_ERR_ALIAS"

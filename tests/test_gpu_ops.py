@@ -100,3 +100,35 @@ def test_backward_op_fp32_grads(gpu):
     assert dA.dtype == torch.float32 and dB.dtype == torch.float32
     assert torch.equal(dX, dX16)
     assert torch.equal(dA.to(torch.bfloat16), dA16) and torch.equal(dB.to(torch.bfloat16), dB16)
+
+
+def test_opcheck_saved_t_ops(gpu):
+    """Schema (including the declared mutation of ``saved``) and fake
+    implementations of lora_linear_train and lora_linear_bwd_saved; Y equals
+    lora_linear's bit for bit."""
+    t = WL.make_layer_inputs(WL.LayerShape(130, 256, 136, 8, 6.0), seed=7, with_dy=True)
+    X, W, A, B, dY = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    torch.library.opcheck(torch.ops.lora_b200.lora_linear_train.default, (X, W, A, B, 0.75),
+                          test_utils=("test_schema", "test_faketensor"))
+    Y, saved = torch.ops.lora_b200.lora_linear_train(X, W, A, B, 0.75)
+    assert torch.equal(Y, torch.ops.lora_b200.lora_linear(X, W, A, B, 0.75))
+    torch.library.opcheck(torch.ops.lora_b200.lora_linear_bwd_saved.default, (X, W, A, B, dY, saved, 0.75),
+                          test_utils=("test_schema", "test_faketensor"))
+
+
+def test_saved_t_backward_op_matches_oracle(gpu):
+    """Y and (dX, dA, dB) of the training pair against the oracle, with and
+    without fp32 gradients."""
+    M, d_in, d_out, r, alpha = 777, 520, 1032, 40, 30.0
+    t = WL.make_layer_inputs(WL.LayerShape(M, d_in, d_out, r, alpha), seed=12, with_dy=True)
+    X, W, A, B, dY = (t[k].cuda() for k in ("X", "W", "A", "B", "dY"))
+    s = alpha / r
+    Y, saved = torch.ops.lora_b200.lora_linear_train(X, W, A, B, s)
+    ref = O.lora_backward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), f64(t["dY"]), alpha)
+    ok, info = lora_tol_check(f64(Y), O.lora_forward(f64(t["X"]), f64(t["W"]), f64(t["A"]), f64(t["B"]), alpha))
+    assert ok, ("Y", info)
+    for fp32 in (False, True):
+        got = torch.ops.lora_b200.lora_linear_bwd_saved(X, W, A, B, dY, saved, s, fp32)
+        for name, g, want in zip(("dX", "dA", "dB"), got, ref):
+            ok, info = lora_tol_check(f64(g.to(torch.bfloat16)), want)
+            assert ok, (name, fp32, info)
