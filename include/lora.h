@@ -97,16 +97,17 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
 
 /*
  * Forward that also keeps T for the backward: Y exactly as lora_fwd (bit for
- * bit), and T = X A^T (unscaled, each value the fp32 sum that the forward's
- * up-projection scales, rounded once to bf16; zero columns past r) written
- * into `workspace`, a buffer of at least lora_bwd_workspace_size(M, d_in,
+ * bit), and T = X A^T (unscaled, an fp32 sum rounded once to bf16; zero
+ * columns past r) written into `workspace`, a buffer of at least lora_bwd_workspace_size(M, d_in,
  * d_out, r) bytes, 256-byte aligned, that overlaps none of X, W, A, B, Y.
  * Pass the same workspace to lora_bwd_ex or lora_bwd_grads with
  * LORA_BWD_T_SAVED, which then skip recomputing T.  The T slot's layout is
  * the library's own; only the workspace as a whole is passed along.
  * In the tiled forward the tile of N index 0 of every M block stores its
- * rows of T from the epilogue (no extra pass over X); in the split-contraction
- * form for small outputs, T is one more launch that reads X.
+ * rows of T from the epilogue (no extra pass over X): each value is the very
+ * sum that the up-projection scales.  In the split-contraction form for
+ * small outputs, T is one more launch that reads X and sums in its own
+ * order.
  * With M == 0 nothing happens (the workspace may then be NULL).
  */
 lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const void* B, void* Y,
