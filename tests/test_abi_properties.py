@@ -1,0 +1,179 @@
+"""Property tests of the host-side argument rules (no GPU): random shapes,
+ranks and pointer layouts through lora_check_args, which validates exactly
+as the entry points do and never launches anything, against a restatement
+of the rules include/lora.h documents:
+
+* NULL   - a required pointer is NULL (X, Y / dY, dX and the workspace may
+           be NULL only when M == 0);
+* SHAPE  - M < 0, d_in or d_out <= 0 or not a multiple of 8, or any of them
+           above 2^30;
+* RANK   - r not a multiple of 8 in [8, 128];
+* ALIGN  - a tensor pointer not 16-byte aligned (the workspace: 256);
+* WORKSPACE - (backward, M > 0) workspace NULL or smaller than required;
+* ALIAS  - an output's byte range overlaps an input's or another output's.
+
+The first rule that fails, in this order, gives the status.  Pointers come
+from a few slots 256 MiB apart plus small offsets, so overlaps and
+misalignment are frequent."""
+import collections
+
+import pytest
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+SLOT = 1 << 28
+BASE = 0x7f0000000000
+LIM = 1 << 30
+
+# statuses the property tests below saw, per entry point (checked at the end)
+SEEN = collections.defaultdict(collections.Counter)
+
+settings.register_profile("abi", max_examples=400, deadline=None, derandomize=True,
+                          suppress_health_check=[HealthCheck.too_slow])
+
+
+def _weighted(common, rare, rare_in=10):
+    """`common` nine times in ten, `rare` otherwise."""
+    return st.integers(0, rare_in - 1).flatmap(lambda k: rare if k == 0 else common)
+
+
+# about one pointer in twenty is NULL; the others sit in one of six slots at
+# offsets that are 16-byte aligned or not and near or far from the slot base
+ptr = st.integers(0, 19).flatmap(
+    lambda k: st.just(0) if k == 0 else st.builds(
+        lambda s, o: BASE + s * SLOT + o, st.integers(0, 5),
+        st.sampled_from([0, 0, 16, 256, 4096, 1 << 20, 1 << 27, 8, 48])))
+dims = _weighted(st.sampled_from([8, 16, 64, 520, 1024, 4096, 14336]),
+                 st.one_of(st.integers(-16, 20000), st.sampled_from([LIM, LIM + 8])))
+rows = _weighted(st.one_of(st.just(0), st.integers(1, 5000)), st.sampled_from([-1, LIM, LIM + 1]))
+ranks = _weighted(st.sampled_from(list(range(8, 129, 8))), st.integers(-1, 140))
+
+
+def _sizes(M, d_in, d_out, r):
+    if M < 0 or d_in <= 0 or d_out <= 0 or d_in % 8 or d_out % 8:
+        return "LORA_ERR_SHAPE"
+    if M > LIM or d_in > LIM or d_out > LIM:
+        return "LORA_ERR_SHAPE"
+    if r < 8 or r > 128 or r % 8:
+        return "LORA_ERR_RANK"
+    return None
+
+
+def _overlap(a, b):
+    (p, n), (q, m) = a, b
+    return n > 0 and m > 0 and p < q + m and q < p + n
+
+
+def _ws_need(M, r):
+    if M == 0:
+        return 0
+    r_pad = (r + 15) // 16 * 16
+    return 2 * ((M * r_pad * 2 + 255) // 256 * 256)
+
+
+def model_fwd(p, M, d_in, d_out, r):
+    X, W, A, B, Y = p
+    for i, q in enumerate(p):
+        if q == 0 and (1 <= i <= 3 or M != 0):
+            return "LORA_ERR_NULL"
+    s = _sizes(M, d_in, d_out, r)
+    if s:
+        return s
+    if any(q % 16 for q in p):
+        return "LORA_ERR_ALIGN"
+    y = (Y, M * d_out * 2)
+    ins = [(X, M * d_in * 2), (W, d_out * d_in * 2), (A, r * d_in * 2), (B, d_out * r * 2)]
+    return "LORA_ERR_ALIAS" if any(_overlap(y, i) for i in ins) else "LORA_OK"
+
+
+def model_bwd(p, M, d_in, d_out, r, ws_bytes):
+    X, W, A, B, dY, dX, dA, dB, ws = p
+    for i, q in enumerate(p[:8]):
+        if q == 0 and (1 <= i <= 3 or i in (6, 7) or M != 0):
+            return "LORA_ERR_NULL"
+    s = _sizes(M, d_in, d_out, r)
+    if s:
+        return s
+    if any(q % 16 for q in p[:8]):
+        return "LORA_ERR_ALIGN"
+    need = _ws_need(M, r)
+    if M > 0:
+        if ws == 0 or ws_bytes < need:
+            return "LORA_ERR_WORKSPACE"
+        if ws % 256:
+            return "LORA_ERR_ALIGN"
+    ins = [(X, M * d_in * 2), (W, d_out * d_in * 2), (A, r * d_in * 2), (B, d_out * r * 2), (dY, M * d_out * 2)]
+    outs = [(dX, M * d_in * 2), (dA, r * d_in * 2), (dB, d_out * r * 2), (ws, need)]
+    for k, o in enumerate(outs):
+        if any(_overlap(o, i) for i in ins) or any(_overlap(o, o2) for o2 in outs[k + 1:]):
+            return "LORA_ERR_ALIAS"
+    return "LORA_OK"
+
+
+def model_merge(p, d_in, d_out, r):
+    W_src, A, B, W_dst = p
+    if any(q == 0 for q in p):
+        return "LORA_ERR_NULL"
+    s = _sizes(0, d_in, d_out, r)
+    if s:
+        return s
+    if any(q % 16 for q in p):
+        return "LORA_ERR_ALIGN"
+    dst = (W_dst, d_out * d_in * 2)
+    if _overlap(dst, (A, r * d_in * 2)) or _overlap(dst, (B, d_out * r * 2)):
+        return "LORA_ERR_ALIAS"
+    if W_dst != W_src and _overlap(dst, (W_src, d_out * d_in * 2)):
+        return "LORA_ERR_ALIAS"
+    return "LORA_OK"
+
+
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=5, max_size=5), M=rows, d_in=dims, d_out=dims, r=ranks)
+def test_forward_rules(built_lib, p, M, d_in, d_out, r):
+    L = built_lib
+    want = model_fwd(p, M, d_in, d_out, r)
+    SEEN["fwd"][want] += 1
+    assert L.STATUS[L.lora_check_args(0, p, M, d_in, d_out, r)] == want
+
+
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=9, max_size=9), M=rows, d_in=dims, d_out=dims, r=ranks,
+       ws_pick=st.sampled_from(["need", "less", "more", "zero"]))
+def test_backward_rules(built_lib, p, M, d_in, d_out, r, ws_pick):
+    L = built_lib
+    need = _ws_need(M, r) if _sizes(M, d_in, d_out, r) is None else 0
+    ws_bytes = {"need": need, "less": max(need - 1, 0), "more": need + 256, "zero": 0}[ws_pick]
+    want = model_bwd(p, M, d_in, d_out, r, ws_bytes)
+    SEEN["bwd"][want] += 1
+    assert L.STATUS[L.lora_check_args(1, p, M, d_in, d_out, r, ws_bytes)] == want
+
+
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=4, max_size=4), d_in=dims, d_out=dims, r=ranks, same=st.booleans())
+def test_merge_rules(built_lib, p, d_in, d_out, r, same):
+    L = built_lib
+    if same:                     # in place: W_dst == W_src is allowed
+        p = [p[0], p[1], p[2], p[0]]
+    want = model_merge(p, d_in, d_out, r)
+    SEEN["merge"][want] += 1
+    assert L.STATUS[L.lora_check_args(2, p, 0, d_in, d_out, r)] == want
+
+
+@pytest.mark.parametrize("M,r", [(1, 8), (300, 24), (4100, 128), (8192, 16), (0, 64)])
+def test_workspace_size_matches_the_documented_layout(built_lib, M, r):
+    assert built_lib.lora_bwd_workspace_size(M, 512, 264, r) == _ws_need(M, r)
+
+
+def test_every_rule_was_reached():
+    """The random cases above reached every status of each entry point at
+    least a few times (runs after them, in file order)."""
+    if not SEEN:
+        pytest.skip("the property tests did not run in this session")
+    expect = {"fwd": {"LORA_OK", "LORA_ERR_NULL", "LORA_ERR_SHAPE", "LORA_ERR_RANK", "LORA_ERR_ALIGN",
+                      "LORA_ERR_ALIAS"},
+              "merge": {"LORA_OK", "LORA_ERR_NULL", "LORA_ERR_SHAPE", "LORA_ERR_RANK", "LORA_ERR_ALIGN",
+                        "LORA_ERR_ALIAS"}}
+    expect["bwd"] = expect["fwd"] | {"LORA_ERR_WORKSPACE"}
+    for op, statuses in expect.items():
+        for s in statuses:
+            assert SEEN[op][s] >= 5, (op, dict(SEEN[op]))
