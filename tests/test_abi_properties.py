@@ -164,9 +164,153 @@ def test_workspace_size_matches_the_documented_layout(built_lib, M, r):
     assert built_lib.lora_bwd_workspace_size(M, 512, 264, r) == _ws_need(M, r)
 
 
+# ------------------------------------------------------------------------
+# The entry points without a lora_check_args op (lora_fwd_save and the
+# two-call backward) are called directly, only with cases that must fail
+# and only on a host without a GPU: there, even a wrong pass stops at the
+# device lookup.  Which of several violated rules is reported is not
+# documented, so the status must be one of the rules the case violates.
+
+try:
+    import torch
+    _HAS_GPU = torch.cuda.is_available()
+except Exception:  # pragma: no cover
+    _HAS_GPU = False
+host_only = pytest.mark.skipif(_HAS_GPU, reason="calls entry points with fake pointers: host without a GPU only")
+
+
+def _viol_bufs(ins, outs):
+    """NULL / ALIGN / ALIAS rules over (ptr, bytes, required) buffers."""
+    v = set()
+    for q, _, req in ins + outs:
+        if q == 0 and req:
+            v.add("LORA_ERR_NULL")
+        if q != 0 and q % 16:
+            v.add("LORA_ERR_ALIGN")
+    for k, (q, n, _) in enumerate(outs):
+        if q == 0:
+            continue
+        if any(p and _overlap((q, n), (p, m)) for p, m, _ in ins) or \
+                any(p and _overlap((q, n), (p, m)) for p, m, _ in outs[k + 1:]):
+            v.add("LORA_ERR_ALIAS")
+    return v
+
+
+def _viol_ws(ws, ws_bytes, need):
+    if need == 0:
+        return set()
+    if ws == 0 or ws_bytes < need:
+        return {"LORA_ERR_WORKSPACE"}
+    return {"LORA_ERR_ALIGN"} if ws % 256 else set()
+
+
+def viol_fwd_save(p, ws, ws_bytes, M, d_in, d_out, r):
+    first = model_fwd(p, M, d_in, d_out, r)
+    if first != "LORA_OK":
+        return {first}           # lora_fwd's own rules come first, in lora_check_args' order
+    need = _ws_need(M, r)
+    v = _viol_ws(ws, ws_bytes, need)
+    if not v and M > 0:
+        X, W, A, B, Y = p
+        sizes = [M * d_in * 2, d_out * d_in * 2, r * d_in * 2, d_out * r * 2, M * d_out * 2]
+        if any(_overlap((ws, need), (q, n)) for q, n in zip(p, sizes)):
+            v.add("LORA_ERR_ALIAS")
+    return v
+
+
+def viol_grads(p, ws, ws_bytes, M, d_in, d_out, r, flags):
+    if flags & ~3:
+        return {"LORA_ERR_FLAGS"}
+    s = _sizes(M, d_in, d_out, r)
+    if s:
+        return {s}
+    gb = 4 if flags & 1 else 2
+    X, A, B, dY, dA, dB = p
+    rows_ = M > 0
+    need = _ws_need(M, r)
+    v = _viol_ws(ws, ws_bytes, need)
+    ins = [(X, M * d_in * 2, rows_), (A, r * d_in * 2, True), (B, d_out * r * 2, True), (dY, M * d_out * 2, rows_)]
+    outs = [(dA, r * d_in * gb, True), (dB, d_out * r * gb, True), (ws if rows_ else 0, need, rows_)]
+    return v | _viol_bufs(ins, outs)
+
+
+def viol_dx(p, ws, ws_bytes, M, d_in, d_out, r):
+    s = _sizes(M, d_in, d_out, r)
+    if s:
+        return {s}
+    W, A, dY, dX = p
+    rows_ = M > 0
+    need = _ws_need(M, r)
+    v = _viol_ws(ws, ws_bytes, need)
+    ins = [(W, d_out * d_in * 2, True), (A, r * d_in * 2, True), (dY, M * d_out * 2, rows_),
+           (ws if rows_ else 0, need, rows_)]
+    outs = [(dX, M * d_in * 2, rows_)]
+    return v | _viol_bufs(ins, outs)
+
+
+def _c(x):
+    import ctypes
+    return ctypes.c_void_p(x) if x else None
+
+
+ws_picks = st.sampled_from(["need", "less", "zero"])
+
+
+def _ws_bytes(pick, M, r, d_in, d_out):
+    need = _ws_need(M, r) if _sizes(M, d_in, d_out, r) is None else 0
+    return {"need": need, "less": max(need - 1, 0), "zero": 0}[pick]
+
+
+@host_only
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=5, max_size=5), ws=ptr, pick=ws_picks, M=rows, d_in=dims, d_out=dims, r=ranks)
+def test_fwd_save_rules(built_lib, p, ws, pick, M, d_in, d_out, r):
+    import ctypes
+    from hypothesis import assume
+    L = built_lib
+    wb = _ws_bytes(pick, M, r, d_in, d_out)
+    v = viol_fwd_save(p, ws, wb, M, d_in, d_out, r)
+    assume(v)
+    SEEN["fwd_save"]["err"] += 1
+    got = L.lib().lora_fwd_save(*[_c(x) for x in p], M, d_in, d_out, r, ctypes.c_float(2.0), _c(ws), wb, None)
+    assert L.STATUS[got] in v, (L.STATUS[got], v)
+
+
+@host_only
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=6, max_size=6), ws=ptr, pick=ws_picks, M=rows, d_in=dims, d_out=dims, r=ranks,
+       flags=st.sampled_from([0, 1, 2, 3, 4, 0x80000000]))
+def test_bwd_grads_rules(built_lib, p, ws, pick, M, d_in, d_out, r, flags):
+    import ctypes
+    from hypothesis import assume
+    L = built_lib
+    wb = _ws_bytes(pick, M, r, d_in, d_out)
+    v = viol_grads(p, ws, wb, M, d_in, d_out, r, flags)
+    assume(v)
+    SEEN["grads"]["err"] += 1
+    got = L.lib().lora_bwd_grads(*[_c(x) for x in p], M, d_in, d_out, r, ctypes.c_float(2.0), _c(ws), wb,
+                                 flags, None)
+    assert L.STATUS[got] in v, (L.STATUS[got], v)
+
+
+@host_only
+@settings(settings.get_profile("abi"))
+@given(p=st.lists(ptr, min_size=4, max_size=4), ws=ptr, pick=ws_picks, M=rows, d_in=dims, d_out=dims, r=ranks)
+def test_bwd_dx_rules(built_lib, p, ws, pick, M, d_in, d_out, r):
+    from hypothesis import assume
+    L = built_lib
+    wb = _ws_bytes(pick, M, r, d_in, d_out)
+    v = viol_dx(p, ws, wb, M, d_in, d_out, r)
+    assume(v)
+    SEEN["dx"]["err"] += 1
+    got = L.lib().lora_bwd_dx(*[_c(x) for x in p], M, d_in, d_out, r, _c(ws), wb, None)
+    assert L.STATUS[got] in v, (L.STATUS[got], v)
+
+
 def test_every_rule_was_reached():
-    """The random cases above reached every status of each entry point at
-    least a few times (runs after them, in file order)."""
+    """The random cases above reached every status of each validator op at
+    least a few times, and the direct entry-point tests ran enough failing
+    cases (runs after them, in file order)."""
     if not SEEN:
         pytest.skip("the property tests did not run in this session")
     expect = {"fwd": {"LORA_OK", "LORA_ERR_NULL", "LORA_ERR_SHAPE", "LORA_ERR_RANK", "LORA_ERR_ALIGN",
@@ -177,3 +321,7 @@ def test_every_rule_was_reached():
     for op, statuses in expect.items():
         for s in statuses:
             assert SEEN[op][s] >= 5, (op, dict(SEEN[op]))
+    if not _HAS_GPU:
+        for op in ("fwd_save", "grads", "dx"):
+            assert SEEN[op]["err"] >= 50, (op, dict(SEEN[op]))
+
