@@ -299,6 +299,40 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
                               size_t workspace_bytes);
 
 /*
+ * Launch plan of a shape (host only: no GPU needed, no device state read,
+ * nothing launched): the kernel configuration the library would choose on a
+ * B200 with `sm_count` SMs, as the entry points choose it (including the
+ * LORA_B200_* overrides in the environment).  For tests and tools; no
+ * computation depends on these fields.  With M == 0 every field is zero.
+ * Returns LORA_ERR_NULL for a NULL `out`, lora_fwd's SHAPE / RANK rules for
+ * the sizes, and LORA_ERR_SHAPE for sm_count outside [2, 4096].
+ */
+typedef struct {
+  int32_t fwd_kind;        /* 0 = tiled kernel (one output tile per CTA or CTA pair),
+                              1 = split contraction (the CTAs of a cluster share a tile) */
+  int32_t fwd_bn;          /* output tile width */
+  int32_t fwd_cg;          /* CTAs per tile (2 = CTA pair) */
+  int32_t fwd_stages;      /* pipeline stages */
+  int32_t fwd_run_l;       /* tiled: 0 = contiguous ranges, L = runs of L N tiles */
+  int32_t fwd_num_m;       /* output tiles along M ... */
+  int32_t fwd_num_n;       /* ... and along N */
+  int32_t fwd_splits;      /* split contraction: CTAs per tile along K (tiled: 1) */
+  uint32_t fwd_smem;       /* dynamic shared memory per CTA, bytes */
+  int32_t bwd1_splits_dt;  /* backward launch 1: contraction splits of the dT job ... */
+  int32_t bwd1_splits_t;   /* ... and of the T job (they share the launch) */
+  int32_t bwd1_saved_splits; /* launch 1 with LORA_BWD_T_SAVED (dT alone) */
+  uint32_t bwd1_smem;      /* launch 1: shared memory per CTA */
+  int32_t bwd2_splits_db;  /* backward launch 2: splits of the dB job ... */
+  int32_t bwd2_splits_da;  /* ... and of the dA job (they share the launch) */
+  uint32_t bwd2_smem;
+  int32_t dx_bn, dx_cg, dx_stages;  /* backward launch 3 (dX), tiled kernel */
+  uint32_t dx_smem;
+  uint64_t workspace_bytes; /* lora_bwd_workspace_size */
+} lora_plan_t;
+
+lora_status_t lora_plan(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int32_t sm_count, lora_plan_t* out);
+
+/*
  * Self-test of the bounded-wait machinery: launches one block that waits on
  * a barrier nothing will arrive on, with the given limit in nanoseconds
  * (clamped to [1e3, 1e9]).  Returns what lora_get_device_status() then

@@ -48,6 +48,17 @@ class _MergeDesc(ctypes.Structure):
                 ("W_dst", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64)]
 
 
+class _Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("fwd_kind", "fwd_bn", "fwd_cg", "fwd_stages", "fwd_run_l",
+                                              "fwd_num_m", "fwd_num_n", "fwd_splits")] + \
+               [("fwd_smem", ctypes.c_uint32)] + \
+               [(n, ctypes.c_int32) for n in ("bwd1_splits_dt", "bwd1_splits_t", "bwd1_saved_splits")] + \
+               [("bwd1_smem", ctypes.c_uint32), ("bwd2_splits_db", ctypes.c_int32),
+                ("bwd2_splits_da", ctypes.c_int32), ("bwd2_smem", ctypes.c_uint32),
+                ("dx_bn", ctypes.c_int32), ("dx_cg", ctypes.c_int32), ("dx_stages", ctypes.c_int32),
+                ("dx_smem", ctypes.c_uint32), ("workspace_bytes", ctypes.c_uint64)]
+
+
 _lib_handle = None
 _lock = threading.Lock()
 
@@ -97,6 +108,8 @@ def lib() -> ctypes.CDLL:
         L.lora_get_device_status.argtypes = []
         L.lora_check_args.restype = ctypes.c_int
         L.lora_check_args.argtypes = [i32, ctypes.POINTER(vp), i32, i64, i64, i64, i32, sz]
+        L.lora_plan.restype = ctypes.c_int
+        L.lora_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan)]
         L.lora_selftest_wait_timeout.restype = ctypes.c_int
         L.lora_selftest_wait_timeout.argtypes = [i64]
         _lib_handle = L
@@ -372,6 +385,14 @@ def lora_check_args(op: int, ptrs: Sequence[int], M: int, d_in: int, d_out: int,
     arr = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(p) if p else None for p in ptrs])
     return int(lib().lora_check_args(int(op), arr, n, int(M), int(d_in), int(d_out), int(r),
                                      int(workspace_bytes)))
+
+
+def lora_plan(M: int, d_in: int, d_out: int, r: int, sm_count: int = 148) -> dict:
+    """The launch plan the library would use for this shape (host only; see
+    include/lora.h), as a dict of lora_plan_t's fields."""
+    out = _Plan()
+    _raise(lib().lora_plan(int(M), int(d_in), int(d_out), int(r), int(sm_count), ctypes.byref(out)), "lora_plan")
+    return {name: int(getattr(out, name)) for name, _ in _Plan._fields_}
 
 
 def lora_selftest_wait_timeout(limit_ns: int) -> int:

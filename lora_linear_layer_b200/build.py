@@ -2,8 +2,9 @@
 
     python -m lora_linear_layer_b200.build [--force]
 
-One translation unit (``csrc/lora_api.cu``) with the kernels included; the
-CUDA runtime is linked statically and the driver's tensor-map encoder is
+Two translation units: ``csrc/lora_api.cu`` (the entry points, with the
+kernels included) and ``csrc/plan_api.cu`` (host-only launch-plan
+introspection); the CUDA runtime is linked statically and the driver's tensor-map encoder is
 looked up at run time, so the library loads on machines without a GPU.
 """
 from __future__ import annotations
@@ -18,6 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(_HERE, "csrc")
 OUT = os.path.join(_HERE, "_lib", "liblora_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "lora.h")
+TRANSLATION_UNITS = ("lora_api.cu", "plan_api.cu")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -48,7 +50,7 @@ def build(force: bool = False, verbose: bool = True, extra_flags=None) -> str:
             return OUT
     os.makedirs(os.path.dirname(OUT), exist_ok=True)
     tmp = OUT + ".tmp"
-    cmd = [nvcc_path()] + NVCC_FLAGS + list(extra_flags or []) + ["-o", tmp, os.path.join(CSRC, "lora_api.cu")]
+    cmd = [nvcc_path()] + NVCC_FLAGS + list(extra_flags or []) + ["-o", tmp] + [os.path.join(CSRC, f) for f in TRANSLATION_UNITS]
     if verbose:
         print("[lora_b200 build]", " ".join(cmd), flush=True)
     subprocess.run(cmd, check=True, cwd=CSRC)

@@ -253,8 +253,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1) merge_kernel(const __grid_co
 }
 
 
+// The plain copy and fill kernels have internal linkage: this header is
+// included by more than one translation unit of the library.
+
 // W_dst <- W_src, 16 bytes per thread per step (restore from pristine).
-__global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+static __global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
   griddep_launch_dependents();
   griddep_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
@@ -262,14 +265,14 @@ __global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__
 }
 
 // Tail of a copy that is not a multiple of 16 bytes (2-byte elements).
-__global__ void copy2_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
+static __global__ void copy2_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
   griddep_launch_dependents();
   griddep_wait();
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (i < n) dst[i] = src[i];
 }
 
-__global__ void zero16_kernel(uint4* __restrict__ dst, size_t n16) {
+static __global__ void zero16_kernel(uint4* __restrict__ dst, size_t n16) {
   griddep_launch_dependents();
   griddep_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)

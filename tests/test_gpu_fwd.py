@@ -104,7 +104,9 @@ TILES = ["256,2", "256,1", "128,2", "128,1"]
 @pytest.mark.parametrize("M,d_in,d_out,r,alpha", [(1000, 1032, 1544, 24, 18.0), (777, 520, 2056, 128, 96.0)])
 def test_fwd_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in, d_out, r, alpha):
     """Every tile configuration (BN, CTA pair or single CTA) and schedule
-    (contiguous ranges, runs of 1 and 3 N tiles) against the oracle."""
+    (contiguous ranges, runs of 1 and 3 N tiles) against the oracle.  At
+    r = 128, 256-wide single-CTA tiles have no room for three stages and the
+    override falls back to the automatic choice (tests/test_plan.py)."""
     monkeypatch.setenv("LORA_B200_FUSED_TILE", tile)
     monkeypatch.setenv("LORA_B200_FUSED_RUN", run)
     sh = WL.LayerShape(M, d_in, d_out, r, alpha)

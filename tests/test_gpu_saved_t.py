@@ -68,13 +68,13 @@ def _fwd_pair(L, d, alpha, ws):
 
 
 SHAPES = [
-    (256, 512, 512, 16, 32.0),      # tiny workload: split-contraction forward
+    (256, 512, 512, 16, 32.0),      # tiny workload (tiled, 128-wide tiles)
     (1, 8, 8, 8, 16.0),
     (300, 520, 264, 8, 6.0),
-    (777, 1032, 1000, 40, 30.0),
+    (777, 1032, 1000, 40, 30.0),    # split-contraction forward: T from one more launch
     (1000, 512, 2056, 64, 128.0),
     (257, 256, 384, 128, 96.0),
-    (2048, 1024, 4096, 32, 64.0),   # tiled forward, CTA pairs
+    (2048, 1024, 4096, 32, 64.0),   # tiled forward, 256-wide tiles, runs of 2
     (4100, 1024, 1536, 32, 64.0),   # ragged last M block
 ]
 
@@ -93,7 +93,8 @@ def test_fwd_save_keeps_y_and_writes_t(gpu, M, d_in, d_out, r, alpha):
 @pytest.mark.parametrize("M,d_in,d_out,r,alpha", [(1000, 1032, 1544, 24, 18.0), (777, 520, 2056, 128, 96.0)])
 def test_fwd_save_every_tile_config_and_schedule(gpu, monkeypatch, tile, run, M, d_in, d_out, r, alpha):
     """The tile of N index 0 of every M block writes T: checked for every tile
-    configuration and schedule (contiguous ranges, runs of 1 and 3)."""
+    configuration and schedule (contiguous ranges, runs of 1 and 3; at
+    r = 128 a forced 256 x 1 tile falls back to the automatic choice)."""
     monkeypatch.setenv("LORA_B200_FUSED_TILE", tile)
     monkeypatch.setenv("LORA_B200_FUSED_RUN", run)
     t, d = _inputs(M, d_in, d_out, r, alpha, seed=7)
