@@ -52,7 +52,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 }
 
 // Warp-converged form for warps that go on to run .sync.aligned tcgen05
-// instructions: lane 0 polls, the verdict is broadcast, and __syncwarp
+// instructions: lane 0 polls, the result is broadcast, and __syncwarp
 // orders the other lanes after lane 0's observation of the barrier.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                   uint64_t limit_ns, uint32_t site, bool cluster_scope = false) {
