@@ -8,7 +8,8 @@
  *
  * its backward for a frozen W (same page, section "BWD kernel speedup",
  * which names the dA, dB and dX kernels; the formulas follow from the
- * forward by the chain rule), with T = X A^T recomputed:
+ * forward by the chain rule), with T = X A^T recomputed (or kept from the
+ * forward through lora_fwd_save and LORA_BWD_T_SAVED):
  *
  *     dT = s dY B,   dB = s dY^T T,   dA = dT^T X,   dX = dY W + dT A
  *
@@ -96,8 +97,9 @@ lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* 
                        void* stream);
 
 /*
- * Forward that also keeps T for the backward: Y exactly as lora_fwd (bit for
- * bit), and T = X A^T (unscaled, an fp32 sum rounded once to bf16; zero
+ * Forward that also keeps T for the backward (the pages describe the forward
+ * and the backward, not what passes between them; keeping T is a choice of
+ * this library): Y exactly as lora_fwd (bit for bit), and T = X A^T (unscaled, an fp32 sum rounded once to bf16; zero
  * columns past r) written into `workspace`, a buffer of at least lora_bwd_workspace_size(M, d_in,
  * d_out, r) bytes, 256-byte aligned, that overlaps none of X, W, A, B, Y.
  * Pass the same workspace to lora_bwd_ex or lora_bwd_grads with
@@ -299,8 +301,8 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
                               size_t workspace_bytes);
 
 /*
- * Launch plan of a shape (host only: no GPU needed, no device state read,
- * nothing launched): the kernel configuration the library would choose on a
+ * Launch plan of a shape (a service of this library, not part of the method;
+ * host only: no GPU needed, no device state read, nothing launched): the kernel configuration the library would choose on a
  * B200 with `sm_count` SMs, as the entry points choose it (including the
  * LORA_B200_* overrides in the environment).  For tests and tools; no
  * computation depends on these fields.  With M == 0 every field is zero.
