@@ -236,3 +236,39 @@ def test_fwd_save_validation(built_lib):
     assert c(X, W, A, B, 0, M, d_in, d_out, r, f, ws, need, None) == "LORA_ERR_NULL"
     assert c(X, W, A, B, Y, M, d_in, d_out, 12, f, ws, need, None) == "LORA_ERR_RANK"
     assert c(X, W, A, B, X, M, d_in, d_out, r, f, ws, need, None) == "LORA_ERR_ALIAS"
+
+
+def _header_structs(path):
+    """{typedef name: [(field, C type)]} for the plain structs of the header
+    (comments removed; several names in one declaration allowed)."""
+    text = re.sub(r"/\*.*?\*/", " ", open(path).read(), flags=re.S)
+    out = {}
+    for body, name in re.findall(r"typedef struct \{(.*?)\}\s*(\w+)\s*;", text, flags=re.S):
+        fields = []
+        for decl in body.split(";"):
+            decl = " ".join(decl.split())
+            if not decl:
+                continue
+            m = re.match(r"((?:const )?[a-z0-9_]+\s*\*?)\s*(.*)", decl)
+            ctype = m.group(1).replace(" ", "")
+            for n in m.group(2).split(","):
+                n = n.strip()
+                if n.startswith("*"):
+                    ctype, n = ctype + "*", n[1:]
+                fields.append((n, ctype))
+        out[name] = fields
+    return out
+
+
+def test_ctypes_structs_mirror_the_header(built_lib):
+    """The binding's ctypes structures have the header structs' fields, in
+    order, with matching types (a mismatch would corrupt every call)."""
+    L = built_lib
+    c = {"constvoid*": ctypes.c_void_p, "void*": ctypes.c_void_p, "int64_t": ctypes.c_int64,
+         "int32_t": ctypes.c_int32, "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64}
+    structs = _header_structs(L.HEADER_PATH)
+    for cname, cls in (("lora_fwd_desc_t", L._FwdDesc), ("lora_merge_desc_t", L._MergeDesc),
+                       ("lora_plan_t", L._Plan)):
+        want = [(n, c[t]) for n, t in structs[cname]]
+        assert [(n, t) for n, t in cls._fields_] == want, cname
+    assert ctypes.sizeof(L._Plan) == 88 and ctypes.sizeof(L._FwdDesc) == 64 and ctypes.sizeof(L._MergeDesc) == 48
