@@ -33,7 +33,8 @@
  *   multiples of any tile size.
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *   asynchronous with respect to the host and ordered on `stream`.
- * - s = alpha / r is computed in fp32 on the host.
+ * - s = alpha / r is computed in fp32 on the host (the *_scaled forms below
+ *   take s itself instead of alpha).
  * - Outputs must not overlap inputs, except W_dst == W_src in lora_merge.
  * - Argument errors are returned before anything is launched and leave no
  *   side effects.  A failed launch returns LORA_ERR_CUDA.  Kernels bound
@@ -58,7 +59,7 @@
 extern "C" {
 #endif
 
-#define LORA_ABI_VERSION 3
+#define LORA_ABI_VERSION 4
 
 typedef enum {
   LORA_OK = 0,
@@ -210,7 +211,8 @@ lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX
  *    with LORA_ERR_WORKSPACE (and a message on stderr) before any launch.
  *  - The first call on each device looks up the array's device address
  *    (with that device current) and keeps it; make that first call before
- *    any stream capture begins.
+ *    any stream capture begins.  After a device reset (a new context) the
+ *    next call looks it up again, so it too should come before a capture.
  *  - All calls share the one array and it keeps the last call's contents;
  *    nothing in it needs to start at zero.  Calls whose work can overlap on
  *    the GPU (e.g. on two streams) race on it: keep them on one stream.
@@ -275,6 +277,44 @@ typedef struct {
 
 lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float alpha,
                                void* stream);
+
+/*
+ * Explicit scale.  Each of these is the entry point of the same name without
+ * "_scaled", with the same arguments, rules and results, except that the
+ * float `scale` takes the place of `alpha` and is used as s itself instead
+ * of s = alpha / r.  rsLoRA is the case in point (unsloth fork commit log,
+ * scripts/benchmarks/qwen3_flex_inference.py: under rsLoRA PEFT keeps
+ * alpha / sqrt(r) in the module's scaling, and that value is what the layer
+ * multiplies by); any other scale (0 gives the base layer alone) works the
+ * same way.  A call with scale == alpha / r computed in fp32 gives the
+ * results of the alpha form bit for bit.
+ *   lora_fwd_scaled            <-> lora_fwd
+ *   lora_fwd_save_scaled       <-> lora_fwd_save
+ *   lora_fwd_batched_scaled    <-> lora_fwd_batched
+ *   lora_bwd_scaled            <-> lora_bwd_ex (flags as there; 0 = lora_bwd)
+ *   lora_bwd_grads_scaled      <-> lora_bwd_grads (lora_bwd_dx takes no scale)
+ *   lora_merge_scaled          <-> lora_merge
+ *   lora_merge_batched_scaled  <-> lora_merge_batched
+ */
+lora_status_t lora_fwd_scaled(const void* X, const void* W, const void* A, const void* B, void* Y,
+                              int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                              void* stream);
+lora_status_t lora_fwd_save_scaled(const void* X, const void* W, const void* A, const void* B, void* Y,
+                                   int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+lora_status_t lora_fwd_batched_scaled(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float scale,
+                                      void* stream);
+lora_status_t lora_bwd_scaled(const void* X, const void* W, const void* A, const void* B,
+                              const void* dY, void* dX, void* dA, void* dB,
+                              int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                              void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
+lora_status_t lora_bwd_grads_scaled(const void* X, const void* A, const void* B, const void* dY, void* dA,
+                                    void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                                    void* workspace, size_t workspace_bytes, uint32_t flags, void* stream);
+lora_status_t lora_merge_scaled(const void* W_src, const void* A, const void* B, void* W_dst,
+                                int64_t d_out, int64_t d_in, int32_t r, float scale, void* stream);
+lora_status_t lora_merge_batched_scaled(const lora_merge_desc_t* descs, int32_t n, int32_t r, float scale,
+                                        void* stream);
 
 /*
  * Restore: W_dst <- W_src, a bit copy of n_elems bf16 values (the pristine

@@ -112,6 +112,14 @@ def lib() -> ctypes.CDLL:
         L.lora_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan)]
         L.lora_selftest_wait_timeout.restype = ctypes.c_int
         L.lora_selftest_wait_timeout.argtypes = [i64]
+        # explicit-scale forms: the same argument lists with `scale` in place of alpha
+        for name, base in (("lora_fwd_scaled", "lora_fwd"), ("lora_fwd_save_scaled", "lora_fwd_save"),
+                           ("lora_fwd_batched_scaled", "lora_fwd_batched"), ("lora_bwd_scaled", "lora_bwd_ex"),
+                           ("lora_bwd_grads_scaled", "lora_bwd_grads"), ("lora_merge_scaled", "lora_merge"),
+                           ("lora_merge_batched_scaled", "lora_merge_batched")):
+            fn = getattr(L, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = list(getattr(L, base).argtypes)
         _lib_handle = L
         return L
 
@@ -177,36 +185,64 @@ def lora_status_string(code: int) -> str:
     return lib().lora_status_string(int(code)).decode()
 
 
-def lora_fwd(X, W, A, B, Y, alpha: float, stream=None) -> None:
-    """Y = X W^T + (alpha/r) (X A^T) B^T (see include/lora.h)."""
+def _fwd_call(name, X, W, A, B, Y, value, stream):
     M, d_in = X.shape
     d_out, r = B.shape
     for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
                     (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
         _check_tensor(t, n, s)
-    code = lib().lora_fwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r,
-                          float(alpha), _stream(stream))
-    _raise(code, "lora_fwd")
+    code = getattr(lib(), name)(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r,
+                                float(value), _stream(stream))
+    _raise(code, name)
+
+
+def lora_fwd(X, W, A, B, Y, alpha: float, stream=None) -> None:
+    """Y = X W^T + (alpha/r) (X A^T) B^T (see include/lora.h)."""
+    _fwd_call("lora_fwd", X, W, A, B, Y, alpha, stream)
+
+
+def lora_fwd_scaled(X, W, A, B, Y, scale: float, stream=None) -> None:
+    """Y = X W^T + scale (X A^T) B^T with the scale given (e.g. rsLoRA's
+    alpha / sqrt(r)); see include/lora.h."""
+    _fwd_call("lora_fwd_scaled", X, W, A, B, Y, scale, stream)
 
 
 def lora_fwd_save(X, W, A, B, Y, alpha: float, workspace, stream=None) -> None:
     """lora_fwd that also writes T = X A^T into the backward's workspace
     (see include/lora.h); pass that workspace to lora_bwd_ex or
     lora_bwd_grads with LORA_BWD_T_SAVED."""
+    _fwd_save_call("lora_fwd_save", X, W, A, B, Y, alpha, workspace, stream)
+
+
+def lora_fwd_save_scaled(X, W, A, B, Y, scale: float, workspace, stream=None) -> None:
+    """lora_fwd_save with the scale given instead of alpha."""
+    _fwd_save_call("lora_fwd_save_scaled", X, W, A, B, Y, scale, workspace, stream)
+
+
+def _fwd_save_call(name, X, W, A, B, Y, value, workspace, stream):
     M, d_in = X.shape
     d_out, r = B.shape
     for t, n, s in ((X, "X", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
                     (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
         _check_tensor(t, n, s)
     ws_bytes = int(workspace.numel() * workspace.element_size())
-    code = lib().lora_fwd_save(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r, float(alpha),
-                               _ptr(workspace), ws_bytes, _stream(stream))
-    _raise(code, "lora_fwd_save")
+    code = getattr(lib(), name)(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out, r, float(value),
+                                _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(code, name)
 
 
 def lora_fwd_batched(items: Sequence[Tuple], alpha: float, stream=None) -> None:
     """One launch for several independent forwards (X, W, A, B, Y) that share
     the rank r and alpha (see include/lora.h)."""
+    _fwd_batched_call("lora_fwd_batched", items, alpha, stream)
+
+
+def lora_fwd_batched_scaled(items: Sequence[Tuple], scale: float, stream=None) -> None:
+    """lora_fwd_batched with the scale given instead of alpha."""
+    _fwd_batched_call("lora_fwd_batched_scaled", items, scale, stream)
+
+
+def _fwd_batched_call(name, items, value, stream):
     n = len(items)
     arr = (_FwdDesc * max(n, 1))()
     r = None
@@ -221,8 +257,8 @@ def lora_fwd_batched(items: Sequence[Tuple], alpha: float, stream=None) -> None:
                           (B, "B", (d_out, r)), (Y, "Y", (M, d_out))):
             _check_tensor(t, nm, sh)
         arr[i] = _FwdDesc(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(Y), M, d_in, d_out)
-    code = lib().lora_fwd_batched(arr, n, int(r or 8), float(alpha), _stream(stream))
-    _raise(code, "lora_fwd_batched")
+    code = getattr(lib(), name)(arr, n, int(r or 8), float(value), _stream(stream))
+    _raise(code, name)
 
 
 def lora_bwd_workspace_size(M: int, d_in: int, d_out: int, r: int) -> int:
@@ -250,6 +286,15 @@ def lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, flags: int 
     """lora_bwd with flags (see include/lora.h).  With LORA_BWD_FP32_GRADS,
     dA and dB are float32 tensors and receive the fp32 reductions that
     lora_bwd would round to bf16."""
+    _bwd_ex_call("lora_bwd_ex", X, W, A, B, dY, dX, dA, dB, alpha, workspace, flags, stream)
+
+
+def lora_bwd_scaled(X, W, A, B, dY, dX, dA, dB, scale: float, workspace, flags: int = 0, stream=None) -> None:
+    """lora_bwd_ex with the scale given instead of alpha."""
+    _bwd_ex_call("lora_bwd_scaled", X, W, A, B, dY, dX, dA, dB, scale, workspace, flags, stream)
+
+
+def _bwd_ex_call(name, X, W, A, B, dY, dX, dA, dB, value, workspace, flags, stream):
     import torch
     M, d_in = X.shape
     d_out, r = B.shape
@@ -263,10 +308,10 @@ def lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, alpha: float, workspace, flags: int 
         if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != s:
             raise ValueError(f"{n} must be a contiguous CUDA tensor of shape {s}")
     ws_bytes = int(workspace.numel() * workspace.element_size())
-    code = lib().lora_bwd_ex(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
-                             M, d_in, d_out, r, float(alpha), _ptr(workspace), ws_bytes, int(flags),
-                             _stream(stream))
-    _raise(code, "lora_bwd_ex")
+    code = getattr(lib(), name)(_ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB),
+                                M, d_in, d_out, r, float(value), _ptr(workspace), ws_bytes, int(flags),
+                                _stream(stream))
+    _raise(code, name)
 
 
 def _check_grads(dA, dB, r: int, d_in: int, d_out: int, flags: int):
@@ -283,15 +328,24 @@ def lora_bwd_grads(X, A, B, dY, dA, dB, alpha: float, workspace, flags: int = 0,
     """First half of the backward (see include/lora.h): T (unless
     LORA_BWD_T_SAVED) and dT into the workspace, then dA and dB.  lora_bwd_dx
     with the same workspace gives dX."""
+    _bwd_grads_call("lora_bwd_grads", X, A, B, dY, dA, dB, alpha, workspace, flags, stream)
+
+
+def lora_bwd_grads_scaled(X, A, B, dY, dA, dB, scale: float, workspace, flags: int = 0, stream=None) -> None:
+    """lora_bwd_grads with the scale given instead of alpha."""
+    _bwd_grads_call("lora_bwd_grads_scaled", X, A, B, dY, dA, dB, scale, workspace, flags, stream)
+
+
+def _bwd_grads_call(name, X, A, B, dY, dA, dB, value, workspace, flags, stream):
     M, d_in = X.shape
     d_out, r = B.shape
     for t, n, s in ((X, "X", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (dY, "dY", (M, d_out))):
         _check_tensor(t, n, s)
     _check_grads(dA, dB, r, d_in, d_out, flags)
     ws_bytes = int(workspace.numel() * workspace.element_size())
-    code = lib().lora_bwd_grads(_ptr(X), _ptr(A), _ptr(B), _ptr(dY), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
-                                float(alpha), _ptr(workspace), ws_bytes, int(flags), _stream(stream))
-    _raise(code, "lora_bwd_grads")
+    code = getattr(lib(), name)(_ptr(X), _ptr(A), _ptr(B), _ptr(dY), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
+                                float(value), _ptr(workspace), ws_bytes, int(flags), _stream(stream))
+    _raise(code, name)
 
 
 def lora_bwd_dx(W, A, dY, dX, workspace, stream=None) -> None:
@@ -325,14 +379,23 @@ def lora_bwd_noalloc(X, W, A, B, dY, dX, dA, dB, alpha: float, stream=None) -> N
 
 def lora_merge(W_src, A, B, W_dst, alpha: float, stream=None) -> None:
     """W_dst = bf16(W_src + (alpha/r) B A); W_dst may be W_src (in place)."""
+    _merge_call("lora_merge", W_src, A, B, W_dst, alpha, stream)
+
+
+def lora_merge_scaled(W_src, A, B, W_dst, scale: float, stream=None) -> None:
+    """W_dst = bf16(W_src + scale B A) with the scale given."""
+    _merge_call("lora_merge_scaled", W_src, A, B, W_dst, scale, stream)
+
+
+def _merge_call(name, W_src, A, B, W_dst, value, stream):
     d_out, d_in = W_src.shape
     r = A.shape[0]
     for t, n, s in ((W_src, "W_src", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
                     (W_dst, "W_dst", (d_out, d_in))):
         _check_tensor(t, n, s)
-    code = lib().lora_merge(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in, r, float(alpha),
-                            _stream(stream))
-    _raise(code, "lora_merge")
+    code = getattr(lib(), name)(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in, r, float(value),
+                                _stream(stream))
+    _raise(code, name)
 
 
 class MergeBatch:
@@ -355,14 +418,25 @@ class MergeBatch:
             self._arr[i] = _MergeDesc(_ptr(W_src), _ptr(A), _ptr(B), _ptr(W_dst), d_out, d_in)
             self._keep.append((W_src, A, B, W_dst))
 
-    def __call__(self, alpha: float, stream=None) -> None:
-        code = lib().lora_merge_batched(self._arr, self.n, self.r, float(alpha), _stream(stream))
-        _raise(code, "lora_merge_batched")
+    def __call__(self, alpha: float, stream=None, *, scale: Optional[float] = None) -> None:
+        """Merge with s = alpha / r, or with s = ``scale`` when it is given
+        (then ``alpha`` is ignored)."""
+        if scale is None:
+            code = lib().lora_merge_batched(self._arr, self.n, self.r, float(alpha), _stream(stream))
+            _raise(code, "lora_merge_batched")
+        else:
+            code = lib().lora_merge_batched_scaled(self._arr, self.n, self.r, float(scale), _stream(stream))
+            _raise(code, "lora_merge_batched_scaled")
 
 
 def lora_merge_batched(items: Sequence[Tuple], r: int, alpha: float, stream=None) -> None:
     """Merge every (W_src, A, B, W_dst) of ``items`` (shared r, alpha)."""
     MergeBatch(items, r)(alpha, stream)
+
+
+def lora_merge_batched_scaled(items: Sequence[Tuple], r: int, scale: float, stream=None) -> None:
+    """lora_merge_batched with the scale given instead of alpha."""
+    MergeBatch(items, r)(0.0, stream, scale=scale)
 
 
 def lora_restore(W_src, W_dst, stream=None) -> None:

@@ -27,7 +27,6 @@ using namespace lora;
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitimate wait
 constexpr uint32_t kSmemMax = 232448;             // 227 KB opt-in dynamic shared memory
-constexpr int kSplitSMs = 148;                    // B200 SM count used to size split-M work
 constexpr uint32_t kSmemPerSM = 233472;           // shared memory per SM (228 KB)
 constexpr uint32_t kBwdFlags = LORA_BWD_FP32_GRADS | LORA_BWD_T_SAVED;  // known backward flag bits
 

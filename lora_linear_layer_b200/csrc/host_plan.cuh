@@ -349,9 +349,11 @@ struct SkinnyCfg {
 // every split keeps at least 4 K blocks.
 // `launch_tiles` is the number of 128-row tiles of the whole launch (both
 // jobs when dB and dA share one), which sets the split count: as many
-// splits as keep every resident CTA slot of the GPU busy, at most 8 (the
-// portable cluster size) and at least 4 K blocks per split.
-void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, int64_t launch_tiles, SkinnyCfg& c) {
+// splits as keep every resident CTA slot of the device's `sm_count` SMs
+// busy, at most 8 (the portable cluster size) and at least 4 K blocks per
+// split.
+void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, int64_t launch_tiles, int sm_count,
+                 SkinnyCfg& c) {
   c.r_pad = r_pad_of(r);
   c.RCW = rcw_of(c.r_pad);
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
@@ -360,7 +362,7 @@ void pick_skinny(int64_t rows, int64_t K, int r, bool r_mn, int out_mode, int64_
   c.smem = L.total + 1024;
   const int per_sm = std::max(1, std::min<int>(int(kSmemPerSM / (c.smem + 1024)),
                                                int(512 / tmem_cols_for(c.r_pad))));
-  const int slots = per_sm * kSplitSMs;
+  const int slots = per_sm * sm_count;
   const int tiles = int(std::max<int64_t>(1, launch_tiles));
   const int nk = int((K + 63) / 64);
   int splits = std::max(1, std::min({slots / tiles, 8, std::max(1, nk / 4)}));
@@ -428,26 +430,36 @@ struct BwdPlan {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, BwdPlan& p) {
+// The backward's workspace: T and dT as bf16 [M, r_pad] each, at 256-byte
+// aligned offsets (independent of the launch plan and of the device).
+struct BwdWorkspace {
+  size_t off_t, off_dt, total;
+};
+
+BwdWorkspace bwd_workspace(int64_t M, int32_t r) {
+  const size_t tb = align256(size_t(M) * size_t(r_pad_of(r)) * 2);
+  return BwdWorkspace{0, tb, 2 * tb};
+}
+
+void plan_bwd(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int sm_count, BwdPlan& p) {
   // dT (contraction d_out) and T (contraction d_in) share the first launch
   // and its split count, which the longer contraction sets for the row
   // tiles of both jobs; the longer job goes first in the grid
   const int64_t both_tiles = 2 * ((M + 127) / 128);
-  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, both_tiles, p.dt_cfg);
-  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, both_tiles, p.t_cfg);
+  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, both_tiles, sm_count, p.dt_cfg);
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, both_tiles, sm_count, p.t_cfg);
   const int s1 = d_out >= d_in ? p.dt_cfg.splits : p.t_cfg.splits;
   resplit_skinny(p.dt_cfg, s1);
   resplit_skinny(p.t_cfg, s1);
-  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, (M + 127) / 128, p.dto_cfg);
+  pick_skinny(M, d_out, r, true, OUT_ROWS_RPAD, (M + 127) / 128, sm_count, p.dto_cfg);
   // dB and dA share one launch, so they share its split count
   const int64_t dbda_tiles = (d_out + 127) / 128 + (d_in + 127) / 128;
-  pick_skinny(d_out, M, r, true, OUT_ROWS_R, dbda_tiles, p.db_cfg);
-  pick_skinny(d_in, M, r, true, OUT_COLS_R, dbda_tiles, p.da_cfg);
-  const int r_pad = r_pad_of(r);
-  const size_t tb = align256(size_t(M) * r_pad * 2);
-  p.off_t = 0;                                         // T   bf16 [M, r_pad]
-  p.off_dt = tb;                                       // dT  bf16 [M, r_pad]
-  p.total = 2 * tb;
+  pick_skinny(d_out, M, r, true, OUT_ROWS_R, dbda_tiles, sm_count, p.db_cfg);
+  pick_skinny(d_in, M, r, true, OUT_COLS_R, dbda_tiles, sm_count, p.da_cfg);
+  const BwdWorkspace w = bwd_workspace(M, r);
+  p.off_t = w.off_t;                                   // T   bf16 [M, r_pad]
+  p.off_dt = w.off_dt;                                 // dT  bf16 [M, r_pad]
+  p.total = w.total;
 }
 
 // -------------------------------------------------------- merge batching ----
@@ -483,7 +495,7 @@ lora_status_t launch_merge_t(const MergeTable& tab, int sm_count, int per_sm, ui
   return launch_ex("merge", kern, dim3(unsigned(grid)), dim3(kMergeThreads), smem, st, nullptr, tab);
 }
 
-lora_status_t run_merge(const MergeItem* items, int n, int32_t r, float alpha, int sm_count, cudaStream_t st) {
+lora_status_t run_merge(const MergeItem* items, int n, int32_t r, float scale, int sm_count, cudaStream_t st) {
   if (n <= 0) return LORA_OK;
   const int r_pad = r_pad_of(r);
   const int rcw = rcw_of(r_pad);
@@ -505,7 +517,7 @@ lora_status_t run_merge(const MergeItem* items, int n, int32_t r, float alpha, i
     tab.r_pad = r_pad;
     tab.n_rchunks = n_rchunks;
     tab.stages = stages;
-    tab.scale = alpha / float(r);
+    tab.scale = scale;
     tab.wait_limit_ns = kWaitLimitNs;
     int tiles = 0, nj = 0;
     for (; i < n && nj < kMergeMaxJobs; ++i) {

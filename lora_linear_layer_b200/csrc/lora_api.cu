@@ -140,9 +140,9 @@ static lora_status_t check_bwd_args(const void* const* ptrs, int32_t n_ptrs, int
 // T = X A^T as bf16 [M, r_pad] (zero columns past r) into `Tws`: one
 // skinny launch.  Arguments already validated, M > 0.
 static lora_status_t launch_t(const void* X, const void* A, int64_t M, int64_t d_in, int32_t r,
-                              __nv_bfloat16* Tws, cudaStream_t st) {
+                              __nv_bfloat16* Tws, int sm_count, cudaStream_t st) {
   SkinnyCfg ct;
-  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, (M + 127) / 128, ct);
+  pick_skinny(M, d_in, r, false, OUT_ROWS_RPAD, (M + 127) / 128, sm_count, ct);
   ct.args.out = Tws;
   CUtensorMap mp, mr;
   if (!make_map(&mp, X, d_in, M, d_in, 64, 128, 128) || !make_map(&mr, A, d_in, r, d_in, 64, ct.r_pad, 128))
@@ -153,7 +153,7 @@ static lora_status_t launch_t(const void* X, const void* A, int64_t M, int64_t d
 // The forward; when `Tws` is not NULL it also receives T = X A^T (bf16
 // [M, r_pad], zero columns past r).  Arguments already validated, M > 0.
 static lora_status_t fwd_run(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
-                             int64_t d_in, int64_t d_out, int32_t r, float alpha, __nv_bfloat16* Tws,
+                             int64_t d_in, int64_t d_out, int32_t r, float scale, __nv_bfloat16* Tws,
                              int sm_count, cudaStream_t st) {
   {
     SplitkPlan pl;
@@ -162,17 +162,17 @@ static lora_status_t fwd_run(const void* X, const void* W, const void* A, const 
       // more (skinny) launch
       SplitkTable<1> t;
       std::memset(&t, 0, sizeof(t));
-      splitk_table_common(t, 1, pl, alpha / float(r));
+      splitk_table_common(t, 1, pl, scale);
       if (!splitk_job(t.job[0], X, W, A, B, Y, M, d_in, d_out, r, pl, 0)) return LORA_ERR_CUDA;
       const int tiles = int(((M + 127) / 128) * ((d_out + 127) / 128));
       const lora_status_t s = launch_splitk(t, tiles, pl, st);
       if (s != LORA_OK || Tws == nullptr) return s;
-      return launch_t(X, A, M, d_in, r, Tws, st);
+      return launch_t(X, A, M, d_in, r, Tws, sm_count, st);
     }
   }
   FusedCfg c;
   if (!pick_fused(M, d_out, d_in, r, false, sm_count, c)) return LORA_ERR_RANK;
-  c.args.scale = alpha / float(r);
+  c.args.scale = scale;
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
   c.args.t_out = Tws;
   CUtensorMap maps[5];
@@ -186,19 +186,32 @@ static lora_status_t fwd_run(const void* X, const void* W, const void* A, const 
   return launch_fused<false>(maps, c, sm_count, st);
 }
 
-lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
-                       int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
+// The forward with the scale given (alpha / r for lora_fwd).
+static lora_status_t fwd_entry(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                               int64_t d_in, int64_t d_out, int32_t r, float scale, void* stream) {
   const void* ptrs[5] = {X, W, A, B, Y};
   lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
   if (s != LORA_OK) return s;
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
   if (M == 0) return LORA_OK;
-  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, alpha, nullptr, dev.sm_count,
+  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, scale, nullptr, dev.sm_count,
                  reinterpret_cast<cudaStream_t>(stream));
 }
 
-lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
+lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                       int64_t d_in, int64_t d_out, int32_t r, float alpha, void* stream) {
+  return fwd_entry(X, W, A, B, Y, M, d_in, d_out, r, alpha / float(r), stream);
+}
+
+lora_status_t lora_fwd_scaled(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                              int64_t d_in, int64_t d_out, int32_t r, float scale, void* stream) {
+  return fwd_entry(X, W, A, B, Y, M, d_in, d_out, r, scale, stream);
+}
+
+// The grouped forward with the scale given (alpha / r for lora_fwd_batched).
+static lora_status_t fwd_batched_entry(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float scale,
+                                       void* stream) {
   if (n < 0) return LORA_ERR_SHAPE;
   if (n == 0) return LORA_OK;
   if (descs == nullptr) return LORA_ERR_NULL;
@@ -240,7 +253,7 @@ lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t 
     if (d.M == 0) continue;
     const int64_t tj = ((d.M + 127) / 128) * ((d.d_out + 127) / 128);
     if (tj >= 4 * int64_t(dev.sm_count) || tj > 65535) {
-      if ((s = lora_fwd(d.X, d.W, d.A, d.B, d.Y, d.M, d.d_in, d.d_out, r, alpha, stream)) != LORA_OK) return s;
+      if ((s = fwd_entry(d.X, d.W, d.A, d.B, d.Y, d.M, d.d_in, d.d_out, r, scale, stream)) != LORA_OK) return s;
     } else {
       group.push_back(i);
     }
@@ -272,32 +285,38 @@ lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t 
       tb += int(((d.M + 127) / 128) * ((d.d_out + 127) / 128));
       ++nj;
     }
-    splitk_table_common(t, nj, pl, alpha / float(r));
+    splitk_table_common(t, nj, pl, scale);
     if ((s = launch_splitk(t, tb, pl, st)) != LORA_OK) return s;
     g = end;
   }
   return LORA_OK;
 }
 
+lora_status_t lora_fwd_batched(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
+  return fwd_batched_entry(descs, n, r, alpha / float(r), stream);
+}
+
+lora_status_t lora_fwd_batched_scaled(const lora_fwd_desc_t* descs, int32_t n, int32_t r, float scale,
+                                      void* stream) {
+  return fwd_batched_entry(descs, n, r, scale, stream);
+}
+
 size_t lora_bwd_workspace_size(int64_t M, int64_t d_in, int64_t d_out, int32_t r) {
   if (check_sizes(M, d_in, d_out, r) != LORA_OK || M == 0) return 0;
-  BwdPlan p;
-  plan_bwd(M, d_in, d_out, r, p);
-  return p.total;
+  return bwd_workspace(M, r).total;
 }
 
 // Launches 1 and 2 of the backward: T (unless `t_saved`: the forward left
 // it in the workspace) and dT into the workspace, then dA and dB.
 // Arguments already validated, M > 0.
 static lora_status_t launch_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA,
-                                      void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
-                                      void* workspace, bool f32, bool t_saved, cudaStream_t st) {
+                                      void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                                      void* workspace, bool f32, bool t_saved, int sm_count, cudaStream_t st) {
   BwdPlan p;
-  plan_bwd(M, d_in, d_out, r, p);
+  plan_bwd(M, d_in, d_out, r, sm_count, p);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_t);
   __nv_bfloat16* dTws = reinterpret_cast<__nv_bfloat16*>(ws + p.off_dt);
-  const float scale = alpha / float(r);
   const int r_pad = r_pad_of(r);
   const int rcw = rcw_of(r_pad);
   lora_status_t s = LORA_OK;
@@ -354,10 +373,8 @@ static lora_status_t launch_bwd_grads(const void* X, const void* A, const void* 
 // Arguments already validated, M > 0.
 static lora_status_t launch_bwd_dx(const void* W, const void* A, const void* dY, void* dX, int64_t M, int64_t d_in,
                                    int64_t d_out, int32_t r, const void* workspace, int sm_count, cudaStream_t st) {
-  BwdPlan p;
-  plan_bwd(M, d_in, d_out, r, p);
-  const __nv_bfloat16* dTws =
-      reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const uint8_t*>(workspace) + p.off_dt);
+  const __nv_bfloat16* dTws = reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const uint8_t*>(workspace) +
+                                                                     bwd_workspace(M, r).off_dt);
   const int r_pad = r_pad_of(r);
   lora_status_t s = LORA_OK;
   // 3. dX = dY W + dT A: one GEMM over the contraction [d_out | r_pad]
@@ -381,7 +398,7 @@ static lora_status_t launch_bwd_dx(const void* W, const void* A, const void* dY,
 // The backward, with `need` bytes of workspace required; `flags` as in
 // lora_bwd_ex.
 static lora_status_t bwd_run(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
-                             void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
+                             void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
                              void* workspace, size_t workspace_bytes, size_t need, uint32_t flags, void* stream) {
   if ((flags & ~kBwdFlags) != 0u) return LORA_ERR_FLAGS;
   const bool f32 = (flags & LORA_BWD_FP32_GRADS) != 0u;
@@ -396,8 +413,8 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
     if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
     return zero_bytes(dB, size_t(d_out) * r * gb, st);
   }
-  if ((s = launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32,
-                            (flags & LORA_BWD_T_SAVED) != 0u, st)) != LORA_OK)
+  if ((s = launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, scale, workspace, f32,
+                            (flags & LORA_BWD_T_SAVED) != 0u, dev.sm_count, st)) != LORA_OK)
     return s;
   return launch_bwd_dx(W, A, dY, dX, M, d_in, d_out, r, workspace, dev.sm_count, st);
 }
@@ -405,7 +422,7 @@ static lora_status_t bwd_run(const void* X, const void* W, const void* A, const 
 lora_status_t lora_bwd(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
                        void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                        void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha / float(r), workspace, workspace_bytes,
                  lora_bwd_workspace_size(M, d_in, d_out, r), 0u, stream);
 }
 
@@ -446,9 +463,10 @@ static lora_status_t check_workspace(const void* workspace, size_t workspace_byt
   return LORA_OK;
 }
 
-lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
-                            int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+// lora_fwd_save with the scale given.
+static lora_status_t fwd_save_entry(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                                    int64_t d_in, int64_t d_out, int32_t r, float scale, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
   const void* ptrs[5] = {X, W, A, B, Y};
   lora_status_t s = lora_check_args(0, ptrs, 5, M, d_in, d_out, r, 0);
   if (s != LORA_OK) return s;
@@ -464,15 +482,27 @@ lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const v
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
   if (M == 0) return LORA_OK;
-  BwdPlan p;
-  plan_bwd(M, d_in, d_out, r, p);
-  __nv_bfloat16* Tws = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(workspace) + p.off_t);
-  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, alpha, Tws, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+  __nv_bfloat16* Tws =
+      reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(workspace) + bwd_workspace(M, r).off_t);
+  return fwd_run(X, W, A, B, Y, M, d_in, d_out, r, scale, Tws, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
-lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
-                             int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
-                             size_t workspace_bytes, uint32_t flags, void* stream) {
+lora_status_t lora_fwd_save(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                            int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return fwd_save_entry(X, W, A, B, Y, M, d_in, d_out, r, alpha / float(r), workspace, workspace_bytes, stream);
+}
+
+lora_status_t lora_fwd_save_scaled(const void* X, const void* W, const void* A, const void* B, void* Y, int64_t M,
+                                   int64_t d_in, int64_t d_out, int32_t r, float scale, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return fwd_save_entry(X, W, A, B, Y, M, d_in, d_out, r, scale, workspace, workspace_bytes, stream);
+}
+
+// lora_bwd_grads with the scale given.
+static lora_status_t bwd_grads_entry(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
+                                     int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale, void* workspace,
+                                     size_t workspace_bytes, uint32_t flags, void* stream) {
   if ((flags & ~kBwdFlags) != 0u) return LORA_ERR_FLAGS;
   lora_status_t s = check_sizes(M, d_in, d_out, r);
   if (s != LORA_OK) return s;
@@ -493,8 +523,21 @@ lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const 
     if ((s = zero_bytes(dA, size_t(r) * d_in * gb, st)) != LORA_OK) return s;
     return zero_bytes(dB, size_t(d_out) * r * gb, st);
   }
-  return launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha, workspace, f32,
-                          (flags & LORA_BWD_T_SAVED) != 0u, st);
+  return launch_bwd_grads(X, A, B, dY, dA, dB, M, d_in, d_out, r, scale, workspace, f32,
+                          (flags & LORA_BWD_T_SAVED) != 0u, dev.sm_count, st);
+}
+
+lora_status_t lora_bwd_grads(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
+                             int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha, void* workspace,
+                             size_t workspace_bytes, uint32_t flags, void* stream) {
+  return bwd_grads_entry(X, A, B, dY, dA, dB, M, d_in, d_out, r, alpha / float(r), workspace, workspace_bytes, flags,
+                         stream);
+}
+
+lora_status_t lora_bwd_grads_scaled(const void* X, const void* A, const void* B, const void* dY, void* dA, void* dB,
+                                    int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale, void* workspace,
+                                    size_t workspace_bytes, uint32_t flags, void* stream) {
+  return bwd_grads_entry(X, A, B, dY, dA, dB, M, d_in, d_out, r, scale, workspace, workspace_bytes, flags, stream);
 }
 
 lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX, int64_t M, int64_t d_in,
@@ -518,21 +561,41 @@ lora_status_t lora_bwd_dx(const void* W, const void* A, const void* dY, void* dX
 lora_status_t lora_bwd_ex(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
                           void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
                           void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
-  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha / float(r), workspace, workspace_bytes,
                  lora_bwd_workspace_size(M, d_in, d_out, r), flags, stream);
 }
 
-lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
-                         int64_t d_in, int32_t r, float alpha, void* stream) {
+lora_status_t lora_bwd_scaled(const void* X, const void* W, const void* A, const void* B, const void* dY, void* dX,
+                              void* dA, void* dB, int64_t M, int64_t d_in, int64_t d_out, int32_t r, float scale,
+                              void* workspace, size_t workspace_bytes, uint32_t flags, void* stream) {
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, scale, workspace, workspace_bytes,
+                 lora_bwd_workspace_size(M, d_in, d_out, r), flags, stream);
+}
+
+// lora_merge with the scale given.
+static lora_status_t merge_entry(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
+                                 int64_t d_in, int32_t r, float scale, void* stream) {
   MergeItem it{W_src, A, B, W_dst, d_out, d_in};
   lora_status_t s = check_merge_item(it, r);
   if (s != LORA_OK) return s;
   DeviceInfo dev;
   if ((s = device_info(dev)) != LORA_OK) return s;
-  return run_merge(&it, 1, r, alpha, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+  return run_merge(&it, 1, r, scale, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
-lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
+lora_status_t lora_merge(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
+                         int64_t d_in, int32_t r, float alpha, void* stream) {
+  return merge_entry(W_src, A, B, W_dst, d_out, d_in, r, alpha / float(r), stream);
+}
+
+lora_status_t lora_merge_scaled(const void* W_src, const void* A, const void* B, void* W_dst, int64_t d_out,
+                                int64_t d_in, int32_t r, float scale, void* stream) {
+  return merge_entry(W_src, A, B, W_dst, d_out, d_in, r, scale, stream);
+}
+
+// lora_merge_batched with the scale given.
+static lora_status_t merge_batched_entry(const lora_merge_desc_t* descs, int32_t n, int32_t r, float scale,
+                                         void* stream) {
   if (n < 0) return LORA_ERR_SHAPE;
   if (n == 0) return LORA_OK;
   if (descs == nullptr) return LORA_ERR_NULL;
@@ -545,7 +608,16 @@ lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int3
   DeviceInfo dev;
   lora_status_t s = device_info(dev);
   if (s != LORA_OK) return s;
-  return run_merge(items.data(), n, r, alpha, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+  return run_merge(items.data(), n, r, scale, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lora_status_t lora_merge_batched(const lora_merge_desc_t* descs, int32_t n, int32_t r, float alpha, void* stream) {
+  return merge_batched_entry(descs, n, r, alpha / float(r), stream);
+}
+
+lora_status_t lora_merge_batched_scaled(const lora_merge_desc_t* descs, int32_t n, int32_t r, float scale,
+                                        void* stream) {
+  return merge_batched_entry(descs, n, r, scale, stream);
 }
 
 lora_status_t lora_restore(const void* W_src, void* W_dst, int64_t n_elems, void* stream) {
@@ -610,8 +682,8 @@ lora_status_t lora_selftest_wait_timeout(int64_t limit_ns) {
 //
 // lora_bwd_noalloc: the backward for callers that cannot call cudaMalloc.
 //
-// lora_bwd needs device scratch (T, dT and the split-M partial sums) and
-// asks the caller for it.  Some callers have no way to provide it: a plugin
+// lora_bwd needs device scratch (the bf16 T and dT of every row, which
+// pass from its first launch to the later ones) and asks the caller for it.  Some callers have no way to provide it: a plugin
 // running inside a host program that owns every device allocation through
 // its own pool, or a service loop that must not allocate once it has
 // started (cudaMalloc can block until the device is idle, and can fail
@@ -625,8 +697,10 @@ lora_status_t lora_selftest_wait_timeout(int64_t limit_ns) {
 // name as a device address (on the host the name refers to a host-side
 // stand-in).  The first call on each device, with that device current,
 // looks the real address up with cudaGetSymbolAddress, checks the result,
-// and keeps it for later calls on that device; that first call should be
-// made before any stream capture begins.  The kernels then receive that
+// and keeps it, with the id of the context it belongs to, for later calls
+// on that device; that first call should be made before any stream capture
+// begins.  After a device reset the next call finds a new context and looks
+// the address up again (it should then also come before any capture).  The kernels then receive that
 // address exactly as they would receive a caller's workspace.
 //
 // All calls share the one array, and it keeps whatever the previous call
@@ -643,25 +717,61 @@ static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[kNoAllocScr
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {};
+struct NoallocAddr {
+  unsigned long long ctx_id;  // the context the address belongs to
+  void* addr;
+};
+NoallocAddr g_noalloc_addr[64] = {};
 
-// Device address of g_bwd_noalloc_scratch on the current device (looked up
-// once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if unknown).  A
+// device reset ends the context and reloads the library's module in the
+// next one at another address; the id tells the two apart, where the
+// context handle itself may be reused.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_cur == nullptr || get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return 0;
+    get_cur = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_bwd_noalloc_scratch in the current device's context,
+// looked up once per context (again after a device reset).
 lora_status_t noalloc_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoallocAddr& e = g_noalloc_addr[dev];
+  if (e.addr == nullptr || ctx == 0 || e.ctx_id != ctx) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch);
+    if (err != cudaSuccess || p == nullptr) {
       std::fprintf(stderr, "lora_bwd_noalloc: cudaGetSymbolAddress failed on device %d: %s\n", dev,
-                   cudaGetErrorString(e));
+                   cudaGetErrorString(err));
+      e.addr = nullptr;
       return LORA_ERR_CUDA;
     }
-    g_noalloc_addr[dev] = p;
+    e.addr = p;
+    e.ctx_id = ctx;
   }
-  *out = g_noalloc_addr[dev];
+  *out = e.addr;
   return LORA_OK;
 }
 }  // namespace
@@ -685,6 +795,7 @@ extern "C" lora_status_t lora_bwd_noalloc(const void* X, const void* W, const vo
     if ((s = device_info(dev)) != LORA_OK) return s;
     if ((s = noalloc_scratch_address(&scratch)) != LORA_OK) return s;
   }
-  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+  return bwd_run(X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, alpha / float(r), scratch,
+                 need > 0 ? kNoAllocScratchBytes : 0,
                  need, 0u, stream);
 }

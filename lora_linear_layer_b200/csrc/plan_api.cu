@@ -55,7 +55,7 @@ lora_status_t lora_plan(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int32
     out->fwd_smem = c.smem;
   }
   BwdPlan p;
-  plan_bwd(M, d_in, d_out, r, p);
+  plan_bwd(M, d_in, d_out, r, sm_count, p);
   out->bwd1_splits_dt = p.dt_cfg.splits;
   out->bwd1_splits_t = p.t_cfg.splits;
   out->bwd1_saved_splits = p.dto_cfg.splits;

@@ -8,15 +8,16 @@ each kernel is a torch.library custom op with a fake implementation, so the
 compiler traces through the layer without a graph break (checked with
 torch._dynamo.explain).  Here:
 
-* ``torch.ops.lora_b200.lora_linear(X, W, A, B, scale)`` runs ``lora_fwd``;
+* ``torch.ops.lora_b200.lora_linear(X, W, A, B, scale)`` runs
+  ``lora_fwd_scaled``;
 * ``torch.ops.lora_b200.lora_linear_bwd(X, W, A, B, dY, scale, fp32_grads)``
-  runs ``lora_bwd_ex`` and returns (dX, dA, dB), dA and dB in fp32 when
+  runs ``lora_bwd_scaled`` and returns (dX, dA, dB), dA and dB in fp32 when
   ``fp32_grads`` (the unrounded reductions, e.g. for fp32 optimizer states
   or a data-parallel sum before rounding), else bf16;
 * ``torch.ops.lora_b200.lora_linear_train(X, W, A, B, scale)`` runs
-  ``lora_fwd_save`` and returns (Y, saved): Y as ``lora_linear`` (bit for
-  bit) and the backward's workspace with T = X A^T already in it; its
-  backward, ``lora_linear_bwd_saved``, runs ``lora_bwd_ex`` with
+  ``lora_fwd_save_scaled`` and returns (Y, saved): Y as ``lora_linear`` (bit
+  for bit) and the backward's workspace with T = X A^T already in it; its
+  backward, ``lora_linear_bwd_saved``, runs ``lora_bwd_scaled`` with
   ``LORA_BWD_T_SAVED`` and so reads X once less (``LoRALinear`` uses this
   pair whenever autograd will need the backward);
 * all have fake (meta) implementations, so they trace under FakeTensorMode
@@ -27,10 +28,9 @@ torch._dynamo.explain).  Here:
 The scale is passed explicitly, so rsLoRA's alpha / sqrt(r) (unsloth fork
 commit log, scripts/benchmarks/qwen3_flex_inference.py: PEFT keeps the
 adapter's scaling, alpha / sqrt(r) under rsLoRA, in the module) is as easy
-to use as alpha / r.  The C ABI takes
-alpha and computes s = alpha / r in fp32; these operators pass
-alpha = scale * r, which gives s exactly when r is a power of two and within
-one fp32 rounding otherwise.
+to use as alpha / r.  The operators call the library's explicit-scale entry
+points (``lora_fwd_scaled``, ``lora_fwd_save_scaled``, ``lora_bwd_scaled``),
+which take s itself (rounded once to fp32) rather than alpha.
 
 Argument marshalling only: all arithmetic runs in the library's kernels.
 """
@@ -41,7 +41,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from . import LORA_BWD_FP32_GRADS, LORA_BWD_T_SAVED, lora_bwd_ex, lora_bwd_workspace_size, lora_fwd, lora_fwd_save
+from . import (LORA_BWD_FP32_GRADS, LORA_BWD_T_SAVED, lora_bwd_scaled, lora_bwd_workspace_size, lora_fwd_save_scaled,
+               lora_fwd_scaled)
 
 _LIB = "lora_b200"
 
@@ -62,7 +63,7 @@ def lora_linear(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.Tens
     """Y = X W^T + scale (X A^T) B^T (bf16, 2-D, contiguous CUDA tensors)."""
     M, d_in, d_out, r = _check(X, W, A, B)
     Y = torch.empty((M, d_out), dtype=X.dtype, device=X.device)
-    lora_fwd(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), Y, scale * r)
+    lora_fwd_scaled(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), Y, scale)
     return Y
 
 
@@ -83,8 +84,8 @@ def lora_linear_bwd(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torch.
     dA = torch.empty((r, d_in), dtype=gdt, device=A.device)
     dB = torch.empty((d_out, r), dtype=gdt, device=B.device)
     ws = torch.empty(max(lora_bwd_workspace_size(M, d_in, d_out, r), 1), dtype=torch.uint8, device=X.device)
-    lora_bwd_ex(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
-                scale * r, ws, LORA_BWD_FP32_GRADS if fp32_grads else 0)
+    lora_bwd_scaled(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
+                    scale, ws, LORA_BWD_FP32_GRADS if fp32_grads else 0)
     return dX, dA, dB
 
 
@@ -115,7 +116,7 @@ def lora_linear_train(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: torc
         raise RuntimeError("lora_linear_train: the library needs a larger workspace than its documented layout")
     Y = torch.empty((M, d_out), dtype=X.dtype, device=X.device)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=X.device)
-    lora_fwd_save(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), Y, scale * r, ws)
+    lora_fwd_save_scaled(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), Y, scale, ws)
     return Y, ws
 
 
@@ -138,8 +139,8 @@ def lora_linear_bwd_saved(X: torch.Tensor, W: torch.Tensor, A: torch.Tensor, B: 
     dA = torch.empty((r, d_in), dtype=gdt, device=A.device)
     dB = torch.empty((d_out, r), dtype=gdt, device=B.device)
     flags = LORA_BWD_T_SAVED | (LORA_BWD_FP32_GRADS if fp32_grads else 0)
-    lora_bwd_ex(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
-                scale * r, saved, flags)
+    lora_bwd_scaled(X.contiguous(), W.contiguous(), A.contiguous(), B.contiguous(), dY.contiguous(), dX, dA, dB,
+                    scale, saved, flags)
     return dX, dA, dB
 
 

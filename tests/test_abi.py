@@ -16,7 +16,7 @@ def test_library_loads_and_exports_every_header_function(built_lib):
     so = L.lib()
     for n in names:
         assert hasattr(so, n), f"{n} declared in include/lora.h but not exported"
-    assert L.lora_abi_version() == 3
+    assert L.lora_abi_version() == 4
 
 
 def test_header_declares_the_hot_path_entry_points(built_lib):

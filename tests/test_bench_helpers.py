@@ -47,3 +47,17 @@ def test_traffic_record_format():
     kernel, workload, h, nbytes = rows[0]
     assert bench.recorded_traffic(kernel, workload, h) == float(nbytes)
     assert bench.recorded_traffic(kernel, workload, "0" * 16) is None
+
+
+def test_peak_follows_the_length_of_the_timed_region():
+    peaks = {"bf16_tflops": 1654.6, "bf16_tflops_sustained": 1410.9}
+    assert bench.pick_peak(peaks, 0.009) == (1654.6, False)       # 20 short steps: burst
+    assert bench.pick_peak(peaks, 0.999) == (1654.6, False)
+    assert bench.pick_peak(peaks, 1.0) == (1410.9, True)          # seconds at the power cap: sustained
+    assert bench.pick_peak({}, 0.01)[0] == bench.FALLBACK_PEAKS["bf16_tflops"]
+
+
+def test_clock_normalised_time():
+    c = bench._clock_normalised(200.0, {"sm_mhz": 1500.0, "sm_max_mhz": 2000.0})
+    assert c["kcycles"] == 300.0 and c["us_at_max_clock"] == 150.0
+    assert bench._clock_normalised(200.0, None) is None

@@ -93,7 +93,8 @@ def test_batched_merge_matches_single_and_restore_cycles_bit_identical(gpu):
         single = torch.empty_like(pristine[i])
         gpu.lora_merge(pristine[i], Ad[i], Bd[i], single, alpha)
         assert torch.equal(single, W_inf[i])
-        _merge_check(m, W_inf[i], r, alpha)
+        info = _merge_check(m, W_inf[i], r, alpha)
+        assert info["max_ulps_noncancel"] <= 1.0 and info["frac_noncancel"] > 0.9, (i, info)
 
     first_state = None
     for cycle in range(10):

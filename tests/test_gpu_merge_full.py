@@ -4,7 +4,8 @@ down 9728->2560), r = 32, alpha = 64, all 252 matrices in one batched call,
 ten perturb + restore + merge refreshes.
 
 Checked: every matrix's rows sampled per 128-row tile against the oracle
-within the merge bound; the pristine copies bit-identical after the ten
+within the merge bound, and within one bf16 ULP on every element whose
+fp32 accumulation does not cancel; the pristine copies bit-identical after the ten
 cycles (SHA-256); each refresh's merged state equal to a second merge of
 the same adapter from pristine, bit for bit."""
 import hashlib
@@ -64,4 +65,6 @@ def test_full_merge_workload(gpu):
                 exact = O.lora_merge(Wr, Af, Bf, alpha)
                 ok, info = merge_tol_check(f64(W_inf[i][rd].cpu()), exact, Wr, Af, Bf, alpha / r)
                 assert ok, (i, shapes[i], info)
+                # one ULP wherever the fp32 accumulation cannot cancel
+                assert info["max_ulps_noncancel"] <= 1.0 and info["frac_noncancel"] > 0.9, (i, shapes[i], info)
     assert [_sha(p) for p in pristine] == h0
