@@ -26,8 +26,12 @@
  *   dY[M, d_out], dX[M, d_in], dA[r, d_in], dB[d_out, r].
  * - All tensor pointers are DEVICE pointers on the current CUDA device,
  *   16-byte aligned.  Pointers to tensors with a zero-sized M dimension
- *   (X, Y, dY, dX, and the workspace) may be NULL when M == 0.  The caller allocates and owns every buffer and the
- *   stream; the library allocates no device memory of its own.
+ *   (X, Y, dY, dX, and the workspace) may be NULL when M == 0.  The caller
+ *   allocates and owns every buffer and the stream; the library never calls
+ *   cudaMalloc.  Its GPU module holds a fixed amount of static device memory
+ *   on every device that loads it: a status word, the forward's exchange
+ *   slots (8 x about 4 MiB, see lora_fwd) and the scratch of
+ *   lora_bwd_noalloc (32 MiB).
  * - d_in and d_out are multiples of 8 (16-byte row pitch); r is a multiple
  *   of 8 in [8, 128]; M >= 0 (M = 0 is a no-op).  Row counts need not be
  *   multiples of any tile size.
@@ -42,8 +46,10 @@
  *   lora_get_device_status() reports (LORA_ERR_TIMEOUT).
  * - Only sm_100 devices (B200) are supported; others get
  *   LORA_ERR_UNSUPPORTED_DEVICE.
- * - Calls on different streams may run concurrently; the library keeps no
- *   per-call state besides the per-device status word.
+ * - Calls on different streams may run concurrently.  Besides the
+ *   per-device status word, the library's only state shared between calls
+ *   is the forward's exchange slots, each bound to one stream (see
+ *   lora_fwd).
  * - Kernels are launched with programmatic dependent launch: a kernel's
  *   set-up may overlap the end of the previous kernel on the stream, but it
  *   touches no global memory before that kernel has completed, so stream
@@ -92,6 +98,16 @@ const char* lora_status_string(lora_status_t status);
  * contraction is split over the CTAs of a thread-block cluster and the
  * partial sums of T and of the base product are added in a fixed order
  * through distributed shared memory (still on chip, no atomics).
+ * Otherwise the tiles are dealt to CTA pairs that walk the output; when
+ * several pairs work on rows of the same M block, the first to compute its
+ * T publishes s T (bf16, the exact operand of the up-projection) in an
+ * exchange slot of library-owned device memory and the others copy it, so
+ * that every pair can be kept busy while T is computed about once per M
+ * block.  A slot is bound to the stream of the first forward that needs
+ * one and serves every later forward on that stream (they run one after
+ * another); up to 8 streams per device get one, and a forward on any other
+ * stream, or one being captured into a CUDA graph, runs without it (slower,
+ * same results).  Y is the same bit for bit with or without the exchange.
  */
 lora_status_t lora_fwd(const void* X, const void* W, const void* A, const void* B, void* Y,
                        int64_t M, int64_t d_in, int64_t d_out, int32_t r, float alpha,
@@ -370,6 +386,10 @@ typedef struct {
   int32_t dx_bn, dx_cg, dx_stages;  /* backward launch 3 (dX), tiled kernel */
   uint32_t dx_smem;
   uint64_t workspace_bytes; /* lora_bwd_workspace_size */
+  int32_t fwd_seeded;      /* tiled: 1 = each cluster first runs fwd_run_l tiles of one M block
+                              (computing its T for all), then the remaining tiles are dealt one at a
+                              time; only with the exchange */
+  int32_t fwd_tx;          /* tiled: 1 = clusters share the down-projection T (the exchange) */
 } lora_plan_t;
 
 lora_status_t lora_plan(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int32_t sm_count, lora_plan_t* out);

@@ -56,7 +56,8 @@ class _Plan(ctypes.Structure):
                [("bwd1_smem", ctypes.c_uint32), ("bwd2_splits_db", ctypes.c_int32),
                 ("bwd2_splits_da", ctypes.c_int32), ("bwd2_smem", ctypes.c_uint32),
                 ("dx_bn", ctypes.c_int32), ("dx_cg", ctypes.c_int32), ("dx_stages", ctypes.c_int32),
-                ("dx_smem", ctypes.c_uint32), ("workspace_bytes", ctypes.c_uint64)]
+                ("dx_smem", ctypes.c_uint32), ("workspace_bytes", ctypes.c_uint64),
+                ("fwd_seeded", ctypes.c_int32), ("fwd_tx", ctypes.c_int32)]
 
 
 _lib_handle = None

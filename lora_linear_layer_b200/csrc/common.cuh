@@ -17,6 +17,7 @@ __device__ unsigned int g_status_info[4] = {0, 0, 0, 0};
 enum WaitSite : uint32_t {
   SITE_FULL = 1, SITE_EMPTY = 2, SITE_VFULL = 3, SITE_VEMPTY = 4, SITE_ACCFULL = 5,
   SITE_ACCEMPTY = 6, SITE_TFULL = 7, SITE_STFULL = 8, SITE_DRAIN = 9, SITE_SELFTEST = 10,
+  SITE_TXMSG = 11, SITE_TXFLAG = 12,
 };
 
 // Wait for the phase of `bar` with the given parity to complete.  Spins on
@@ -47,6 +48,30 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
         __threadfence();
         return false;
       }
+    }
+  }
+}
+
+// Wait until the global word `p` reads `want` (acquire at GPU scope), with
+// the same limit and give-up behaviour as wait_bounded.
+__device__ __forceinline__ bool wait_word_bounded(const uint32_t* p, uint32_t want, volatile int* abort_flag,
+                                                  uint64_t limit_ns, uint32_t site) {
+  if (ld_acquire_gpu(p) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) == want) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      if (atomicOr(&g_status, 1u) == 0u) {
+        g_status_info[0] = blockIdx.x + (blockIdx.y << 16);
+        g_status_info[1] = threadIdx.x;
+        g_status_info[2] = site;
+        g_status_info[3] = want;
+      }
+      __threadfence();
+      return false;
     }
   }
 }

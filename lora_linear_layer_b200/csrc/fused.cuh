@@ -48,6 +48,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "texchange.cuh"
 
 namespace lora {
 
@@ -69,6 +70,9 @@ struct FusedArgs {
   int32_t num_m, num_n;     // tile counts (M tiles of 128 * CG rows)
   int32_t band_w, n_bands;  // column bands of the schedule
   int32_t run_l;            // 0: contiguous ranges; L > 0: runs of L N-tiles dealt round-robin
+  int32_t seeded;           // with run_l: 0 = runs cover every N tile; 1 = one seeding run of run_l
+                            // tiles per cluster, then every other tile round-robin (see TileSched)
+  TxSlot* tx;               // forward: exchange slot the clusters share T through (texchange.cuh), or NULL
   uint64_t wait_limit_ns;
 };
 
@@ -105,21 +109,66 @@ struct FusedLayout {
 //    M-major, are dealt round-robin to the clusters: the tiles in flight at
 //    any time cover only ~G*run_l/num_n M blocks (compact L2 footprint),
 //    and T is computed once per run.
+//  run_l > 0, seeded: two phases, for launches whose clusters share T
+//    through the exchange (texchange.cuh).  Seeding: cluster c runs
+//    run_l N tiles of M block c % num_m from N tile run_l * (c / num_m),
+//    so every M block's T is computed (and published) at the start, by at
+//    least one cluster when there are at least num_m clusters.  Then every
+//    tile the seeding left over, M-major, is dealt round-robin, as in the
+//    dX form: the tiles in flight cover only a few M blocks and every W
+//    tile, the operands stay in L2, and each of these tiles copies its
+//    M block's s T instead of computing it.
 struct TileSched {
   int num_m, num_n, band_w, n_bands, run_l, G, c;
   int band, t, t_end, band_n0, w;
   int runs_per_m, run, run_end, run_pos, run_len, run_m, run_n0;
+  // seeded schedule: first-class blocks (m < r0) and their leftover tiles
+  // per block, the other blocks' count, the next round-robin index, total
+  int seeded, r0, c_hi, c_lo, rr_i, rr_end;
+  bool main_done;
   __device__ TileSched(const FusedArgs& a, int G_, int c_)
       : num_m(a.num_m), num_n(a.num_n), band_w(a.band_w), n_bands(a.n_bands), run_l(a.run_l), G(G_), c(c_),
         band(-1), t(0), t_end(0), band_n0(0), w(1), runs_per_m(1), run(0), run_end(0), run_pos(0), run_len(0),
-        run_m(0), run_n0(0) {
-    if (run_l > 0) {
+        run_m(0), run_n0(0), seeded(a.seeded), r0(0), c_hi(0), c_lo(0), rr_i(0), rr_end(0), main_done(false) {
+    if (run_l > 0 && seeded) {
+      // clusters with c % num_m == m seed M block m: a(m) runs of run_l
+      const int a_lo = G / num_m;
+      r0 = G % num_m;  // blocks m < r0 have a_lo + 1 seeding runs
+      c_hi = num_n - imin(num_n, (a_lo + 1) * run_l);
+      c_lo = num_n - imin(num_n, a_lo * run_l);
+      rr_i = c;
+      rr_end = r0 * c_hi + (num_m - r0) * c_lo;
+    } else if (run_l > 0) {
       runs_per_m = (num_n + run_l - 1) / run_l;
       run = c - G;
       run_end = num_m * runs_per_m;
     }
   }
   __device__ bool next(int& m, int& n) {
+    if (run_l > 0 && seeded) {
+      if (!main_done) {
+        // the seeding run (empty when it would start past the last N tile)
+        const int n0 = run_l * (c / num_m);
+        if (run_pos < imin(run_l, num_n - n0)) {
+          m = c % num_m;
+          n = n0 + run_pos++;
+          return true;
+        }
+        main_done = true;
+      }
+      if (rr_i >= rr_end) return false;
+      const int i = rr_i;
+      rr_i += G;
+      if (i < r0 * c_hi) {
+        m = i / c_hi;
+        n = num_n - c_hi + i % c_hi;
+      } else {
+        const int j = i - r0 * c_hi;
+        m = r0 + j / c_lo;
+        n = num_n - c_lo + j % c_lo;
+      }
+      return true;
+    }
     if (run_l > 0) {
       if (run_pos >= run_len) {
         run += G;
@@ -226,8 +275,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const uint32_t tfull = bar0 + 8u * (2 * S + 4);
   const uint32_t stfull = bar0 + 8u * (2 * S + 5);
   const uint32_t drain = bar0 + 8u * (2 * S + 6);
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_bar + 8 * (2 * S + 7));
+  const uint32_t txbar = bar0 + 8u * (2 * S + 7);      // a T tile's mode message is in tx_msg
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_bar + 8 * (2 * S + 8));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // T tile mode message from the MMA thread to the epilogues of both CTAs:
+  // 1 = copy s T from the exchange, 0 = compute it
+  volatile uint32_t* const tx_msg = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+  // from the (leader's) producer to the MMA thread, published by its arrive
+  // on a T tile's first stage: each T tile's mode, in a ring (the producer
+  // runs at most `stages` stages, so fewer than 8 T tiles, ahead)
+  volatile uint8_t* const tx_mode = reinterpret_cast<volatile uint8_t*>(tmem_slot + 3);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -246,6 +303,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     mbar_init(tfull, 1);
     mbar_init(stfull, 4 * CG);
     mbar_init(drain, 1);
+    mbar_init(txbar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -283,17 +341,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int n_clusters = int(gridDim.x) / CG;
   const int cluster_id = int(blockIdx.x) / CG;
   const int u_rows = a.r_pad / CG;        // U rows held by this CTA
+  const uint32_t tx_full = (1u << (4 * CG)) - 1u;  // every epilogue warp of the cluster has published
+  TxSlot* const tx = MN ? nullptr : a.tx;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
     if (lane == 0) {
       TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, ntp = 0;
       bool ok = true;
       while (ok && sch.next(m, n)) {
         const bool ttile = !MN && (m != prev_m);
         prev_m = m;
+        if (ttile && leader) {
+          // copy s T when another cluster has published this M block's
+          // (checked here, a few stages ahead of the MMA thread)
+          tx_mode[ntp & 7u] = tx != nullptr && ld_acquire_gpu(&tx->flags[m]) == tx_full ? 1 : 0;
+          ++ntp;
+        }
         const uint32_t bytes = L.p_bytes + L.q_bytes + (ttile ? L.u_bytes : 0u);
         const int row0 = m * (kBM * CG) + int(rank) * kBM;
         const int qrow0 = n * BN + int(rank) * BNC;
@@ -365,11 +431,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       while (ok && sch.next(m, n)) {
         const bool ttile = !MN && (m != prev_m);
         prev_m = m;
+        // A T tile copies s T from the exchange when the producer found this
+        // M block's published, else computes T; both CTAs' epilogues are
+        // told which (the previous T tile's message has been read: its
+        // stfull wait came after).  The producer's choice is visible once
+        // the tile's first stage is full.
+        bool tload = false;
+        if (ttile) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL, kClusterScope)) break;
+          tload = tx_mode[ntt & 7u] != 0;
+          const uint32_t msg = tload ? 1u : 0u;
+          *tx_msg = msg;
+          if constexpr (CG > 1) {
+            st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<uint32_t*>(tx_msg)), 1u), msg);
+            mbar_arrive_cluster(mapa_shared(txbar, 1u));
+          }
+          mbar_arrive(txbar);
+        }
+        const bool tcomp = ttile && !tload;
         const uint32_t b = tcount & 1u;
         if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY, kClusterScope))
           break;
         uint32_t t_col = kFold ? b * acc_stride + BN : 2u * BN;
-        if (ttile && borrow) {
+        if (tcomp && borrow) {
           const uint32_t ob = b ^ 1u;
           if (!wait_bounded(accempty0 + 8u * ob, next_acc_parity(ob), abort_flag, lim, SITE_ACCEMPTY,
                             kClusterScope))
@@ -419,7 +503,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
           return true;
         };
-        ok = ttile ? k_loop(std::true_type{}) : k_loop(std::false_type{});
+        ok = tcomp ? k_loop(std::true_type{}) : k_loop(std::false_type{});
         if (!ok) break;
         if (MN) {
           G::commit_all(accfull0 + 8u * b);
@@ -427,7 +511,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           continue;
         }
         if (ttile) {
-          G::commit_all(tfull);
+          if (tcomp) G::commit_all(tfull);
           if (!wait_bounded(stfull, ntt & 1u, abort_flag, lim, SITE_STFULL, kClusterScope)) break;
           ++ntt;
         }
@@ -458,7 +542,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const uint32_t lane_base = uint32_t(q * 32) << 16;
     TileSched sch(a, n_clusters, cluster_id);
     int m, n, prev_m = -1;
-    uint32_t ntt = 0, tcount = 0;
+    uint32_t ntt = 0, ntc = 0, tcount = 0;  // T tiles; T tiles that computed T
     uint32_t full_waits0 = 0u, full_waits1 = 0u;  // completed accfull waits per buffer
     uint8_t* const st_ptr = gbase + L.off_st;
     // this warp's output staging buffers (used in turn when there are two)
@@ -469,41 +553,78 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       prev_m = m;
       const uint32_t b = tcount & 1u;
       if (ttile) {
-        if (!warp_wait_bounded(tfull, ntt & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
+        // the MMA thread's message: compute T (and publish it) or copy it
+        if (!warp_wait_bounded(txbar, ntt & 1u, abort_flag, lim, SITE_TXMSG, kClusterScope)) break;
         ++ntt;
-        tc_fence_after();
-        const uint32_t t_col = kFold ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
+        const bool tload = (*tx_msg & 1u) != 0u;
         const int t_row = m * (kBM * CG) + int(rank) * kBM + row;
-        __nv_bfloat16* const t_dst =
-            a.t_out != nullptr && n == 0 && t_row < a.M ? a.t_out + size_t(t_row) * size_t(a.r_pad) : nullptr;
-        for (int col = 0; col < a.r_pad; col += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(tmem + lane_base + t_col + uint32_t(col), v);
-          tmem_ld_wait();
-          if (t_dst != nullptr) {
-            uint32_t tu[8];
+        if (!tload) {
+          if (!warp_wait_bounded(tfull, ntc & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
+          ++ntc;
+          tc_fence_after();
+          const uint32_t t_col = kFold ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
+          // every tile that computes T stores it for the backward when asked
+          // (the same values whichever tile of the M block does)
+          __nv_bfloat16* const t_dst =
+              a.t_out != nullptr && t_row < a.M ? a.t_out + size_t(t_row) * size_t(a.r_pad) : nullptr;
+          __nv_bfloat16* const x_dst = tx != nullptr ? tx->t + size_t(t_row) * size_t(a.r_pad) : nullptr;
+          for (int col = 0; col < a.r_pad; col += 16) {
+            uint32_t v[16];
+            tmem_ld_x16(tmem + lane_base + t_col + uint32_t(col), v);
+            tmem_ld_wait();
+            if (t_dst != nullptr) {
+              uint32_t tu[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) tu[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* d = reinterpret_cast<uint4*>(t_dst + col);
-            d[0] = make_uint4(tu[0], tu[1], tu[2], tu[3]);
-            d[1] = make_uint4(tu[4], tu[5], tu[6], tu[7]);
+              for (int i = 0; i < 8; ++i)
+                tu[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              uint4* d = reinterpret_cast<uint4*>(t_dst + col);
+              d[0] = make_uint4(tu[0], tu[1], tu[2], tu[3]);
+              d[1] = make_uint4(tu[4], tu[5], tu[6], tu[7]);
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * a.scale, __uint_as_float(v[2 * i + 1]) * a.scale);
+            const uint4 lo = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            const uint4 hi = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            const int c = col / RCW;
+            const int cin = (col % RCW) / 8;  // 16-byte chunk inside the rank row
+            uint8_t* chunk = st_ptr + c * (kBM * kRSpan);
+            *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin, kRSpan)) = lo;
+            *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin + 1, kRSpan)) = hi;
+            if (x_dst != nullptr) {
+              uint4* d = reinterpret_cast<uint4*>(x_dst + col);
+              d[0] = lo;
+              d[1] = hi;
+            }
           }
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * a.scale, __uint_as_float(v[2 * i + 1]) * a.scale);
-          const int c = col / RCW;
-          const int cin = (col % RCW) / 8;  // 16-byte chunk inside the rank row
-          uint8_t* chunk = st_ptr + c * (kBM * kRSpan);
-          *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin, kRSpan)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin + 1, kRSpan)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if (tx != nullptr) {
+            // publish: this warp's 32 rows of s T are in the exchange
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atom_or_release_gpu(&tx->flags[m], 1u << (int(rank) * 4 + q));
+          }
+        } else {
+          // another cluster published this M block's s T (the MMA thread saw
+          // its flag complete): copy this thread's row into shared memory
+          if (!wait_word_bounded(&tx->flags[m], tx_full, abort_flag, lim, SITE_TXFLAG)) break;
+          const __nv_bfloat16* const src = tx->t + size_t(t_row) * size_t(a.r_pad);
+          for (int col = 0; col < a.r_pad; col += 16) {
+            const uint4 lo = ld_global_cg_v4(src + col);
+            const uint4 hi = ld_global_cg_v4(src + col + 8);
+            const int c = col / RCW;
+            const int cin = (col % RCW) / 8;
+            uint8_t* chunk = st_ptr + c * (kBM * kRSpan);
+            *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin, kRSpan)) = lo;
+            *reinterpret_cast<uint4*>(chunk + swz_offset(row, cin + 1, kRSpan)) = hi;
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           G::arrive_leader(stfull);
-          if (borrow) G::arrive_leader(accempty0 + 8u * (b ^ 1u));
+          if (borrow && !tload) G::arrive_leader(accempty0 + 8u * (b ^ 1u));
         }
       }
       const uint32_t fpar = (b ? full_waits1++ : full_waits0++) & 1u;
@@ -562,6 +683,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     __syncwarp();
     tc_fence_after();
     G::dealloc(tmem, 512);
+  }
+  if (warp == 0 && leader && tx != nullptr) {
+    // every role of both CTAs is done with the exchange slot
+    __syncwarp();
+    tx_finish(tx, n_clusters, a.num_m, lane);
   }
 }
 

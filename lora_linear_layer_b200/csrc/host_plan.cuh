@@ -35,6 +35,10 @@ using namespace lora;
 struct FusedCfg {
   int BN, CG, RCW, r_pad, n_rchunks, stages, ep_bufs;
   uint32_t smem;
+  bool tx_fits;              // forward whose T fits an exchange slot (and the exchange is enabled)
+  int seeded_l;              // seeded schedule's run length when the launch gets a slot (0: runs) ...
+  double seeded_cost;
+  int run_l_plain;           // ... and the run length without one (runs cover every N tile)
   FusedArgs args;
 };
 
@@ -58,6 +62,13 @@ void tile_override(int& BN, int& CG) {
     BN = b;
     CG = g;
   }
+}
+
+// LORA_B200_TX=0 turns the forward's T exchange between clusters off (every
+// tile that starts an M block then computes T itself); for tests.
+bool tx_enabled() {
+  const char* e = std::getenv("LORA_B200_TX");
+  return !(e != nullptr && e[0] == '0');
 }
 
 // Optional schedule override from LORA_B200_FUSED_RUN (-1 = choose).
@@ -161,8 +172,48 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
       best_cost = cost;
     }
   }
+  a.seeded = 0;
+  a.tx = nullptr;             // the launch assigns a slot
+  // The T exchange (texchange.cuh): a cluster starting on an M block whose
+  // T another cluster has published copies it instead of computing it.
+  // That allows the seeded schedule (TileSched): every cluster first runs
+  // L tiles of one M block, which computes and publishes every block's T;
+  // the rest is dealt round-robin like the dX form's single tiles, whose
+  // operands stay in L2 (8192 x 4096 x 4096: dX read 114 MB from DRAM, the
+  // forward's runs of 8 on 64 of 74 clusters 312 MB) and which keeps every
+  // cluster busy.  Used when every M block gets a seeding run, the operands
+  // need one column band (they fit L2) and the model (L + 0.5 tile times
+  // for the seeding run, 3% per copying tile after it) beats the runs.
+  c.tx_fits = !mn && num_m <= int(kTxMaxBlocks) &&
+              double(num_m) * double(kBM * c.CG) * double(c.r_pad) <= double(kTxElems) && tx_enabled();
+  c.seeded_l = 0;
+  c.seeded_cost = 0.0;
+  if (c.tx_fits && best_l > 0 && a.n_bands == 1 && clusters >= num_m) {
+    for (int l = 2; l <= 4; ++l) {
+      const int64_t a_lo = clusters / num_m, r0 = clusters % num_m;
+      const int64_t seeded = r0 * std::min<int64_t>(num_n, (a_lo + 1) * l) +
+                             (num_m - r0) * std::min<int64_t>(num_n, a_lo * l);
+      const int64_t rest = int64_t(num_m) * num_n - seeded;
+      const double cost = l + 0.5 + double((rest + clusters - 1) / clusters) * 1.03;
+      // shorter seeding runs keep more tiles in the L2-friendly order: a
+      // longer one must be clearly cheaper in the model
+      if (cost < best_cost - 0.25 && (c.seeded_l == 0 || cost < c.seeded_cost - 0.15)) {
+        c.seeded_l = l;
+        c.seeded_cost = cost;
+      }
+    }
+  }
+  // LORA_B200_SEEDED_L=L forces the seeded schedule's run length (when the
+  // schedule applies at all); for tests and measurements
+  if (const char* e = std::getenv("LORA_B200_SEEDED_L")) {
+    const int l = std::atoi(e);
+    if (c.seeded_l > 0 && l >= 1 && l <= num_n) c.seeded_l = l;
+  }
   const int ro = run_override();
-  a.run_l = ro >= 0 ? ro : best_l;
+  if (ro >= 0) c.seeded_l = 0;
+  c.run_l_plain = ro >= 0 ? ro : best_l;
+  a.run_l = c.seeded_l > 0 ? c.seeded_l : c.run_l_plain;
+  a.seeded = c.seeded_l > 0 ? 1 : 0;
   a.wait_limit_ns = kWaitLimitNs;
   return true;
 }

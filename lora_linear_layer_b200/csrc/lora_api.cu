@@ -44,6 +44,96 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
 
 }  // namespace lora
 
+namespace {
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if unknown).  A
+// device reset ends the context and reloads the library's module in the
+// next one at another address; the id tells the two apart, where the
+// context handle itself may be reused.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_cur == nullptr || get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return 0;
+    get_cur = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// The forward's T exchange slots (texchange.cuh) of each device.  Each slot
+// is bound to one stream, by the stream's unique id, the first time a
+// launch on that stream asks for one, and stays bound to it.  Launches on
+// one stream run one after the other (every kernel of this library waits
+// for the previous kernel of its stream to complete before it touches
+// global memory), so a slot is never used by two launches at once and each
+// launch finds it as the previous one left it: clean.  A stream that finds
+// every slot bound to other streams runs without the exchange, and so does
+// a launch being captured into a graph (a replay could run at any time,
+// beside the slot's stream).
+struct TxPool {
+  unsigned long long ctx_id = 0;
+  TxSlot* base = nullptr;
+  unsigned long long stream_id[kTxSlots] = {};  // bound stream's id + 1; 0 = unbound
+};
+std::mutex g_txpool_mu;
+TxPool g_txpool[64];
+
+// The exchange slot of stream `st` on the current device, or NULL.
+TxSlot* tx_slot_for(cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return nullptr;
+  unsigned long long sid = 0;
+  if (cudaStreamGetId(st, &sid) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const unsigned long long ctx = current_ctx_id();
+  if (ctx == 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_txpool_mu);
+  TxPool& p = g_txpool[dev];
+  if (p.base == nullptr || p.ctx_id != ctx) {
+    // first use in this context (again after a device reset): the slots' address
+    void* b = nullptr;
+    if (cudaGetSymbolAddress(&b, g_tx) != cudaSuccess || b == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    p.base = reinterpret_cast<TxSlot*>(b);
+    p.ctx_id = ctx;
+    for (int i = 0; i < kTxSlots; ++i) p.stream_id[i] = 0;
+  }
+  for (int i = 0; i < kTxSlots; ++i)
+    if (p.stream_id[i] == sid + 1) return p.base + i;
+  for (int i = 0; i < kTxSlots; ++i)
+    if (p.stream_id[i] == 0) {
+      p.stream_id[i] = sid + 1;
+      return p.base + i;
+    }
+  return nullptr;
+}
+
+}  // namespace
+
 // ================================================================ C ABI ====
 
 extern "C" {
@@ -175,6 +265,12 @@ static lora_status_t fwd_run(const void* X, const void* W, const void* A, const 
   c.args.scale = scale;
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
   c.args.t_out = Tws;
+  // with an exchange slot, the schedule that shares T between clusters
+  TxSlot* const tx = c.tx_fits ? tx_slot_for(st) : nullptr;
+  c.args.tx = tx;
+  const bool seeded = tx != nullptr && c.seeded_l > 0;
+  c.args.run_l = seeded ? c.seeded_l : c.run_l_plain;
+  c.args.seeded = seeded ? 1 : 0;
   CUtensorMap maps[5];
   const uint32_t bnc = uint32_t(c.BN / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
@@ -722,34 +818,6 @@ struct NoallocAddr {
   void* addr;
 };
 NoallocAddr g_noalloc_addr[64] = {};
-
-typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
-typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
-
-// Unique id of the calling thread's current context (0 if unknown).  A
-// device reset ends the context and reloads the library's module in the
-// next one at another address; the id tells the two apart, where the
-// context handle itself may be reused.
-unsigned long long current_ctx_id() {
-  static CtxGetCurrentFn get_cur = nullptr;
-  static CtxGetIdFn get_id = nullptr;
-  if (get_cur == nullptr || get_id == nullptr) {
-    void* f1 = nullptr;
-    void* f2 = nullptr;
-    cudaDriverEntryPointQueryResult q1, q2;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
-        q1 != cudaDriverEntryPointSuccess ||
-        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
-        q2 != cudaDriverEntryPointSuccess)
-      return 0;
-    get_cur = reinterpret_cast<CtxGetCurrentFn>(f1);
-    get_id = reinterpret_cast<CtxGetIdFn>(f2);
-  }
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
-  return id;
-}
 
 // Device address of g_bwd_noalloc_scratch in the current device's context,
 // looked up once per context (again after a device reset).

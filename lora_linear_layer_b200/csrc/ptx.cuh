@@ -342,6 +342,45 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 
 namespace lora {
 
+// 32-bit global load with acquire semantics at GPU scope.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// atomic OR with release semantics at GPU scope.
+__device__ __forceinline__ void atom_or_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// 32-bit atomic add with acquire-release semantics at GPU scope; returns
+// the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// 32-bit store into another CTA's shared memory (shared::cluster address).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// 16-byte global load cached in L2 only (never a stale L1 line).
+__device__ __forceinline__ uint4 ld_global_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+}  // namespace lora
+
+namespace lora {
+
 // 16-byte load from another CTA's shared memory (shared::cluster address).
 __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t cluster_addr) {
   float4 v;

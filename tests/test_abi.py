@@ -271,4 +271,4 @@ def test_ctypes_structs_mirror_the_header(built_lib):
                        ("lora_plan_t", L._Plan)):
         want = [(n, c[t]) for n, t in structs[cname]]
         assert [(n, t) for n, t in cls._fields_] == want, cname
-    assert ctypes.sizeof(L._Plan) == 88 and ctypes.sizeof(L._FwdDesc) == 64 and ctypes.sizeof(L._MergeDesc) == 48
+    assert ctypes.sizeof(L._Plan) == 96 and ctypes.sizeof(L._FwdDesc) == 64 and ctypes.sizeof(L._MergeDesc) == 48

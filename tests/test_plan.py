@@ -16,6 +16,66 @@ DS = [8, 64, 136, 520, 1024, 4096, 14336, 16384]
 RS = [8, 16, 24, 32, 40, 64, 96, 128]
 
 
+def schedule_tiles(p, G):
+    """Every (m, n) tile the clusters 0..G-1 take under the run schedule of a
+    plan (run_l > 0), restated from the kernel's tile schedule.  Runs: runs
+    of run_l N tiles of one M block dealt round-robin.  Seeded: cluster c
+    first runs run_l tiles of M block c % num_m from N tile
+    run_l * (c // num_m); every tile no seeding run covers is then dealt
+    round-robin in M-major order."""
+    num_m, num_n, L = p["fwd_num_m"], p["fwd_num_n"], p["fwd_run_l"]
+    out = []
+    if p["fwd_seeded"]:
+        covered = set()
+        for c in range(G):
+            n0 = L * (c // num_m)
+            run = [(c % num_m, n) for n in range(n0, min(n0 + L, num_n))]
+            out.append(run)
+            covered.update(run)
+        rest = [(m, n) for m in range(num_m) for n in range(num_n) if (m, n) not in covered]
+        for c in range(G):
+            out[c] = out[c] + rest[c::G]
+        return [t for per in out for t in per]
+    rpm = -(-num_n // L)
+    for c in range(G):
+        for run in range(c, num_m * rpm, G):
+            m, n0 = run // rpm, (run % rpm) * L
+            out += [(m, n) for n in range(n0, min(n0 + L, num_n))]
+    return out
+
+
+def test_seeded_schedule_covers_every_tile_once_for_any_cluster_count():
+    """The kernel learns its cluster count at launch (it may differ from the
+    planned one); the seeded schedule must still cover every tile exactly
+    once.  The closed-form index map of the kernel (two classes of M block
+    by their number of seeding runs) is checked against the plain
+    enumeration above."""
+    for num_m, num_n, L in ((32, 16, 2), (32, 16, 4), (64, 16, 2), (5, 9, 3), (1, 3, 2), (7, 40, 2), (3, 2, 4)):
+        p = dict(fwd_num_m=num_m, fwd_num_n=num_n, fwd_run_l=L, fwd_seeded=1)
+        want = [(m, n) for m in range(num_m) for n in range(num_n)]
+        for G in (1, 2, 3, num_m - 1, num_m, num_m + 1, 2 * num_m + 3, 74, 200):
+            if G < 1:
+                continue
+            assert sorted(schedule_tiles(p, G)) == want, (num_m, num_n, L, G)
+            # the kernel's closed form for the round-robin part
+            a_lo, r0 = G // num_m, G % num_m
+            c_hi = num_n - min(num_n, (a_lo + 1) * L)
+            c_lo = num_n - min(num_n, a_lo * L)
+            covered = set()
+            for c in range(G):
+                n0 = L * (c // num_m)
+                covered.update((c % num_m, n) for n in range(n0, min(n0 + L, num_n)))
+            rest = [(m, n) for m in range(num_m) for n in range(num_n) if (m, n) not in covered]
+            assert r0 * c_hi + (num_m - r0) * c_lo == len(rest)
+            for i, t in enumerate(rest):
+                if i < r0 * c_hi:
+                    m, n = i // c_hi, num_n - c_hi + i % c_hi
+                else:
+                    j = i - r0 * c_hi
+                    m, n = r0 + j // c_lo, num_n - c_lo + j % c_lo
+                assert (m, n) == t, (num_m, num_n, L, G, i)
+
+
 def _no_empty_split(nk, s):
     return s == 1 or (s - 1) * math.ceil(nk / s) < nk
 
@@ -32,9 +92,16 @@ def _check_plan(p, M, d_in, d_out, r, forced_tile=None, forced_run=None):
         if forced_tile:
             assert (p["fwd_bn"], p["fwd_cg"]) == forced_tile, where
         if forced_run is not None:
-            assert p["fwd_run_l"] == forced_run, where
-        else:
+            assert p["fwd_run_l"] == forced_run and p["fwd_seeded"] == 0, where
+        elif p["fwd_seeded"] == 0:
             assert p["fwd_run_l"] == 0 or 1 <= p["fwd_run_l"] <= min(p["fwd_num_n"], 8), where
+        else:
+            # seeded: only with the T exchange and a seeding run for every M block
+            assert p["fwd_tx"] == 1 and 2 <= p["fwd_run_l"] <= 4, where
+            assert p["fwd_num_m"] <= 148 // p["fwd_cg"], where
+            if p["fwd_num_m"] * p["fwd_num_n"] <= 4096:
+                assert sorted(schedule_tiles(p, 148 // p["fwd_cg"])) == \
+                    [(m, n) for m in range(p["fwd_num_m"]) for n in range(p["fwd_num_n"])], where
     else:
         assert p["fwd_kind"] == 1 and forced_tile is None, where
         assert p["fwd_bn"] == 128 and p["fwd_cg"] == 1 and p["fwd_stages"] >= 1, where
@@ -55,7 +122,7 @@ def _check_plan(p, M, d_in, d_out, r, forced_tile=None, forced_run=None):
 
 @pytest.mark.parametrize("r", RS)
 def test_every_plan_fits_and_covers(built_lib, monkeypatch, r):
-    for v in ("LORA_B200_FUSED_TILE", "LORA_B200_FUSED_RUN", "LORA_B200_SPLITK"):
+    for v in ("LORA_B200_FUSED_TILE", "LORA_B200_FUSED_RUN", "LORA_B200_SPLITK", "LORA_B200_TX", "LORA_B200_SEEDED_L"):
         monkeypatch.delenv(v, raising=False)
     for M, d_in, d_out in itertools.product(MS, DS, DS):
         _check_plan(built_lib.lora_plan(M, d_in, d_out, r), M, d_in, d_out, r)
@@ -68,7 +135,7 @@ def test_forced_tiles_fit(built_lib, monkeypatch, tile):
     single-CTA tiles at r = 128: they leave room for two stages, the planner
     wants three for 256-wide tiles, and the override falls back to the
     automatic choice for the shape."""
-    for v in ("LORA_B200_FUSED_RUN", "LORA_B200_SPLITK"):
+    for v in ("LORA_B200_FUSED_RUN", "LORA_B200_SPLITK", "LORA_B200_TX", "LORA_B200_SEEDED_L"):
         monkeypatch.delenv(v, raising=False)
     for r, M, d in itertools.product(RS, (1, 1000, 8192), (64, 1032, 4096)):
         monkeypatch.delenv("LORA_B200_FUSED_TILE", raising=False)
@@ -104,13 +171,14 @@ def test_forced_split_contraction(built_lib, monkeypatch):
 
 def test_named_workloads(built_lib, monkeypatch):
     """The launch configurations the benchmark and the documentation name."""
-    for v in ("LORA_B200_FUSED_TILE", "LORA_B200_FUSED_RUN", "LORA_B200_SPLITK"):
+    for v in ("LORA_B200_FUSED_TILE", "LORA_B200_FUSED_RUN", "LORA_B200_SPLITK", "LORA_B200_TX", "LORA_B200_SEEDED_L"):
         monkeypatch.delenv(v, raising=False)
-    p = built_lib.lora_plan(8192, 4096, 4096, 16)       # attention projection
-    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"]) == (0, 256, 2, 8)
+    p = built_lib.lora_plan(8192, 4096, 4096, 16)       # attention projection: seeded, runs of 2
+    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_seeded"], p["fwd_tx"]) == \
+        (0, 256, 2, 2, 1, 1)
     assert (p["dx_bn"], p["dx_cg"]) == (256, 2)
     p = built_lib.lora_plan(16384, 4096, 14336, 64)     # MLP up-projection
-    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"]) == (0, 256, 2, 7)
+    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_seeded"]) == (0, 256, 2, 7, 0)
     p = built_lib.lora_plan(128, 4096, 4096, 16)        # weight-streaming: split contraction
     assert (p["fwd_kind"], p["fwd_splits"]) == (1, 4)
     assert all(v == 0 for v in built_lib.lora_plan(0, 512, 264, 16).values())
