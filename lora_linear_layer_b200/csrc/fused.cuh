@@ -113,31 +113,38 @@ struct FusedLayout {
 //    through the exchange (texchange.cuh).  Seeding: cluster c runs
 //    run_l N tiles of M block c % num_m from N tile run_l * (c / num_m),
 //    so every M block's T is computed (and published) at the start, by at
-//    least one cluster when there are at least num_m clusters.  Then every
-//    tile the seeding left over, M-major, is dealt round-robin, as in the
-//    dX form: the tiles in flight cover only a few M blocks and every W
-//    tile, the operands stay in L2, and each of these tiles copies its
-//    M block's s T instead of computing it.
+//    least one cluster when there are at least num_m clusters (the seeding
+//    stays inside the first column band).  Then every tile the seeding left
+//    over is dealt round-robin, band by band and M-major inside a band, as
+//    in the dX form: the tiles in flight cover only a few M blocks and the
+//    W tiles of one band, the operands stay in L2, and each of these tiles
+//    copies its M block's s T instead of computing it.
 struct TileSched {
   int num_m, num_n, band_w, n_bands, run_l, G, c;
   int band, t, t_end, band_n0, w;
   int runs_per_m, run, run_end, run_pos, run_len, run_m, run_n0;
   // seeded schedule: first-class blocks (m < r0) and their leftover tiles
-  // per block, the other blocks' count, the next round-robin index, total
-  int seeded, r0, c_hi, c_lo, rr_i, rr_end;
+  // per block in the first band (w0 wide), the other blocks' count, the
+  // first band's leftover total, the next round-robin index, the total
+  int seeded, r0, c_hi, c_lo, w0, p0, rr_i, rr_end;
   bool main_done;
   __device__ TileSched(const FusedArgs& a, int G_, int c_)
       : num_m(a.num_m), num_n(a.num_n), band_w(a.band_w), n_bands(a.n_bands), run_l(a.run_l), G(G_), c(c_),
         band(-1), t(0), t_end(0), band_n0(0), w(1), runs_per_m(1), run(0), run_end(0), run_pos(0), run_len(0),
-        run_m(0), run_n0(0), seeded(a.seeded), r0(0), c_hi(0), c_lo(0), rr_i(0), rr_end(0), main_done(false) {
+        run_m(0), run_n0(0), seeded(a.seeded), r0(0), c_hi(0), c_lo(0), w0(0), p0(0), rr_i(0), rr_end(0),
+        main_done(false) {
     if (run_l > 0 && seeded) {
       // clusters with c % num_m == m seed M block m: a(m) runs of run_l
+      // (the host keeps every seeding run inside the first band; the kernel
+      // clips a run at the last N tile in any case)
       const int a_lo = G / num_m;
       r0 = G % num_m;  // blocks m < r0 have a_lo + 1 seeding runs
-      c_hi = num_n - imin(num_n, (a_lo + 1) * run_l);
-      c_lo = num_n - imin(num_n, a_lo * run_l);
+      w0 = imin(band_w, num_n);
+      c_hi = w0 - imin(w0, (a_lo + 1) * run_l);
+      c_lo = w0 - imin(w0, a_lo * run_l);
       rr_i = c;
-      rr_end = r0 * c_hi + (num_m - r0) * c_lo;
+      p0 = r0 * c_hi + (num_m - r0) * c_lo;
+      rr_end = p0 + num_m * (num_n - w0);
     } else if (run_l > 0) {
       runs_per_m = (num_n + run_l - 1) / run_l;
       run = c - G;
@@ -159,13 +166,20 @@ struct TileSched {
       if (rr_i >= rr_end) return false;
       const int i = rr_i;
       rr_i += G;
-      if (i < r0 * c_hi) {
+      if (i < r0 * c_hi) {  // first band, blocks with one more seeding run
         m = i / c_hi;
-        n = num_n - c_hi + i % c_hi;
-      } else {
+        n = w0 - c_hi + i % c_hi;
+      } else if (i < p0) {  // first band, the other blocks
         const int j = i - r0 * c_hi;
         m = r0 + j / c_lo;
-        n = num_n - c_lo + j % c_lo;
+        n = w0 - c_lo + j % c_lo;
+      } else {              // later bands, whole, M-major (only the last may be narrower)
+        const int j = i - p0;
+        const int b = 1 + j / (num_m * band_w);
+        const int jb = j - (b - 1) * num_m * band_w;
+        const int wb = imin(band_w, num_n - b * band_w);
+        m = jb / wb;
+        n = b * band_w + jb % wb;
       }
       return true;
     }

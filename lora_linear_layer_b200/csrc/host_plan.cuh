@@ -181,18 +181,20 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   // the rest is dealt round-robin like the dX form's single tiles, whose
   // operands stay in L2 (8192 x 4096 x 4096: dX read 114 MB from DRAM, the
   // forward's runs of 8 on 64 of 74 clusters 312 MB) and which keeps every
-  // cluster busy.  Used when every M block gets a seeding run, the operands
-  // need one column band (they fit L2) and the model (L + 0.5 tile times
-  // for the seeding run, 3% per copying tile after it) beats the runs.
+  // cluster busy.  Used when every M block gets a seeding run inside the
+  // first column band and the model (L + 0.5 tile times for the seeding
+  // run, 3% per copying tile after it) beats the runs.
   c.tx_fits = !mn && num_m <= int(kTxMaxBlocks) &&
               double(num_m) * double(kBM * c.CG) * double(c.r_pad) <= double(kTxElems) && tx_enabled();
   c.seeded_l = 0;
   c.seeded_cost = 0.0;
-  if (c.tx_fits && best_l > 0 && a.n_bands == 1 && clusters >= num_m) {
+  if (c.tx_fits && best_l > 0 && clusters >= num_m) {
     for (int l = 2; l <= 4; ++l) {
       const int64_t a_lo = clusters / num_m, r0 = clusters % num_m;
-      const int64_t seeded = r0 * std::min<int64_t>(num_n, (a_lo + 1) * l) +
-                             (num_m - r0) * std::min<int64_t>(num_n, a_lo * l);
+      const int64_t w0 = std::min(a.band_w, num_n);
+      if ((a_lo + (r0 > 0 ? 1 : 0)) * l > w0) continue;  // the seeding stays inside the first band
+      const int64_t seeded = r0 * std::min<int64_t>(w0, (a_lo + 1) * l) +
+                             (num_m - r0) * std::min<int64_t>(w0, a_lo * l);
       const int64_t rest = int64_t(num_m) * num_n - seeded;
       const double cost = l + 0.5 + double((rest + clusters - 1) / clusters) * 1.03;
       // shorter seeding runs keep more tiles in the L2-friendly order: a

@@ -26,6 +26,7 @@ SHAPES = [
     (16384, 4096, 4096, 24, 18.0, None),     # 64 M blocks for 74 pairs, r = 24 -> 32
     (8000, 1032, 4104, 40, 30.0, None),      # ragged M, N and K
     (4100, 1024, 6152, 16, 12.0, "128,1"),   # 128-wide single CTAs: T folded into the base product
+    (8192, 8192, 8192, 16, 32.0, None),      # four column bands: the tiles after seeding go band by band
 ]
 
 

@@ -24,6 +24,7 @@ def schedule_tiles(p, G):
     run_l * (c // num_m); every tile no seeding run covers is then dealt
     round-robin in M-major order."""
     num_m, num_n, L = p["fwd_num_m"], p["fwd_num_n"], p["fwd_run_l"]
+    bw = p.get("band_w", num_n)
     out = []
     if p["fwd_seeded"]:
         covered = set()
@@ -32,7 +33,8 @@ def schedule_tiles(p, G):
             run = [(c % num_m, n) for n in range(n0, min(n0 + L, num_n))]
             out.append(run)
             covered.update(run)
-        rest = [(m, n) for m in range(num_m) for n in range(num_n) if (m, n) not in covered]
+        rest = [(m, n) for b0 in range(0, num_n, bw) for m in range(num_m)
+                for n in range(b0, min(b0 + bw, num_n)) if (m, n) not in covered]
         for c in range(G):
             out[c] = out[c] + rest[c::G]
         return [t for per in out for t in per]
@@ -50,30 +52,43 @@ def test_seeded_schedule_covers_every_tile_once_for_any_cluster_count():
     once.  The closed-form index map of the kernel (two classes of M block
     by their number of seeding runs) is checked against the plain
     enumeration above."""
-    for num_m, num_n, L in ((32, 16, 2), (32, 16, 4), (64, 16, 2), (5, 9, 3), (1, 3, 2), (7, 40, 2), (3, 2, 4)):
-        p = dict(fwd_num_m=num_m, fwd_num_n=num_n, fwd_run_l=L, fwd_seeded=1)
+    cases = ((32, 16, 2, 16), (32, 16, 4, 16), (64, 16, 2, 16), (5, 9, 3, 9), (1, 3, 2, 3), (7, 40, 2, 40),
+             (3, 2, 4, 2), (64, 56, 2, 19), (32, 32, 2, 9), (5, 23, 2, 6), (9, 17, 3, 17))
+    for num_m, num_n, L, bw in cases:
+        p = dict(fwd_num_m=num_m, fwd_num_n=num_n, fwd_run_l=L, fwd_seeded=1, band_w=bw)
         want = [(m, n) for m in range(num_m) for n in range(num_n)]
         for G in (1, 2, 3, num_m - 1, num_m, num_m + 1, 2 * num_m + 3, 74, 200):
             if G < 1:
                 continue
-            assert sorted(schedule_tiles(p, G)) == want, (num_m, num_n, L, G)
-            # the kernel's closed form for the round-robin part
             a_lo, r0 = G // num_m, G % num_m
-            c_hi = num_n - min(num_n, (a_lo + 1) * L)
-            c_lo = num_n - min(num_n, a_lo * L)
+            if (a_lo + (r0 > 0)) * L > min(bw, num_n):
+                continue                                   # the host keeps the seeding in the first band
+            assert sorted(schedule_tiles(p, G)) == want, (num_m, num_n, L, bw, G)
+            # the kernel's closed form for the round-robin part
+            w0 = min(bw, num_n)
+            c_hi = w0 - min(w0, (a_lo + 1) * L)
+            c_lo = w0 - min(w0, a_lo * L)
+            p0 = r0 * c_hi + (num_m - r0) * c_lo
             covered = set()
             for c in range(G):
                 n0 = L * (c // num_m)
                 covered.update((c % num_m, n) for n in range(n0, min(n0 + L, num_n)))
-            rest = [(m, n) for m in range(num_m) for n in range(num_n) if (m, n) not in covered]
-            assert r0 * c_hi + (num_m - r0) * c_lo == len(rest)
+            rest = [(m, n) for b0 in range(0, num_n, bw) for m in range(num_m)
+                    for n in range(b0, min(b0 + bw, num_n)) if (m, n) not in covered]
+            assert p0 + num_m * (num_n - w0) == len(rest)
             for i, t in enumerate(rest):
                 if i < r0 * c_hi:
-                    m, n = i // c_hi, num_n - c_hi + i % c_hi
-                else:
+                    m, n = i // c_hi, w0 - c_hi + i % c_hi
+                elif i < p0:
                     j = i - r0 * c_hi
-                    m, n = r0 + j // c_lo, num_n - c_lo + j % c_lo
-                assert (m, n) == t, (num_m, num_n, L, G, i)
+                    m, n = r0 + j // c_lo, w0 - c_lo + j % c_lo
+                else:
+                    j = i - p0
+                    b = 1 + j // (num_m * bw)
+                    jb = j - (b - 1) * num_m * bw
+                    wb = min(bw, num_n - b * bw)
+                    m, n = jb // wb, b * bw + jb % wb
+                assert (m, n) == t, (num_m, num_n, L, bw, G, i)
 
 
 def _no_empty_split(nk, s):
@@ -178,7 +193,7 @@ def test_named_workloads(built_lib, monkeypatch):
         (0, 256, 2, 2, 1, 1)
     assert (p["dx_bn"], p["dx_cg"]) == (256, 2)
     p = built_lib.lora_plan(16384, 4096, 14336, 64)     # MLP up-projection
-    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_seeded"]) == (0, 256, 2, 7, 0)
+    assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_seeded"]) == (0, 256, 2, 2, 1)
     p = built_lib.lora_plan(128, 4096, 4096, 16)        # weight-streaming: split contraction
     assert (p["fwd_kind"], p["fwd_splits"]) == (1, 4)
     assert all(v == 0 for v in built_lib.lora_plan(0, 512, 264, 16).values())
