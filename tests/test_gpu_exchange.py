@@ -128,3 +128,32 @@ def test_exchange_two_streams_at_once(gpu, monkeypatch):
         assert gpu.lora_get_device_status() == 0
         for i in (0, 1):
             assert torch.equal(Ys[i], want[i]), i
+
+
+def test_forward_captured_in_a_graph_runs_without_the_exchange_same_bits(gpu, monkeypatch):
+    """A forward captured into a CUDA graph gets no exchange slot (a replay
+    may run at any time beside the slot's stream) and runs the plain run
+    schedule; replayed, it gives the eager forward's Y bit for bit."""
+    _env(monkeypatch)
+    M, d_in, d_out, r, alpha = 8192, 4096, 4096, 16, 32.0
+    t = WL.make_layer_inputs(WL.LayerShape(M, d_in, d_out, r, alpha), seed=41)
+    X, W, A, B = (dev(t[k]) for k in ("X", "W", "A", "B"))
+    want = run_fwd(gpu, t["X"], t["W"], t["A"], t["B"], alpha)
+    Y = torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        gpu.lora_fwd(X, W, A, B, Y, alpha)          # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    Y.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gpu.lora_fwd(X, W, A, B, Y, alpha)
+    for _ in range(2):
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y, want)
+    del g
+    assert gpu.lora_get_device_status() == 0
