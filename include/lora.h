@@ -389,7 +389,8 @@ typedef struct {
   int32_t fwd_seeded;      /* tiled: 1 = each cluster first runs fwd_run_l tiles of one M block
                               (computing its T for all), then the remaining tiles are dealt one at a
                               time; only with the exchange */
-  int32_t fwd_tx;          /* tiled: 1 = clusters share the down-projection T (the exchange) */
+  int32_t fwd_tx;          /* tiled: 1 = clusters share the down-projection T (the exchange; with the
+                              seeded schedule only) */
 } lora_plan_t;
 
 lora_status_t lora_plan(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int32_t sm_count, lora_plan_t* out);

@@ -257,7 +257,11 @@ struct Group<2> {
   static __device__ __forceinline__ void cluster_sync() { cluster_barrier_sync(); }
 };
 
-template <int BN, bool MN, int RCW, int CG>
+// TX: the forward with an exchange slot (texchange.cuh); its steps are
+// compiled only into these instances, so a launch without a slot runs a
+// kernel with none of them (a smaller kernel: the tiny forward measured
+// 1-2 us slower with the exchange code compiled in but not taken).
+template <int BN, bool MN, int RCW, int CG, bool TX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_lora_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
@@ -265,6 +269,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(CG == 1 || CG == 2, "CG");
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
+  static_assert(!(TX && MN), "the exchange is a forward feature");
   constexpr bool kQmn = MN;             // Q read MN-major
   using G = Group<CG>;
   constexpr int BNC = BN / CG;          // Q / V rows held by this CTA
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int cluster_id = int(blockIdx.x) / CG;
   const int u_rows = a.r_pad / CG;        // U rows held by this CTA
   const uint32_t tx_full = (1u << (4 * CG)) - 1u;  // every epilogue warp of the cluster has published
-  TxSlot* const tx = MN ? nullptr : a.tx;
+  TxSlot* const tx = TX ? a.tx : nullptr;  // a compile-time NULL without TX
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
@@ -368,10 +373,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       while (ok && sch.next(m, n)) {
         const bool ttile = !MN && (m != prev_m);
         prev_m = m;
-        if (ttile && leader) {
+        if (ttile && leader && tx != nullptr) {
           // copy s T when another cluster has published this M block's
           // (checked here, a few stages ahead of the MMA thread)
-          tx_mode[ntp & 7u] = tx != nullptr && ld_acquire_gpu(&tx->flags[m]) == tx_full ? 1 : 0;
+          tx_mode[ntp & 7u] = ld_acquire_gpu(&tx->flags[m]) == tx_full ? 1 : 0;
           ++ntp;
         }
         const uint32_t bytes = L.p_bytes + L.q_bytes + (ttile ? L.u_bytes : 0u);
@@ -450,8 +455,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // told which (the previous T tile's message has been read: its
         // stfull wait came after).  The producer's choice is visible once
         // the tile's first stage is full.
+        // (launches without an exchange slot take none of these steps)
         bool tload = false;
-        if (ttile) {
+        if (ttile && tx != nullptr) {
           if (!wait_bounded(full_bar(stage), phase, abort_flag, lim, SITE_FULL, kClusterScope)) break;
           tload = tx_mode[ntt & 7u] != 0;
           const uint32_t msg = tload ? 1u : 0u;
@@ -568,9 +574,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint32_t b = tcount & 1u;
       if (ttile) {
         // the MMA thread's message: compute T (and publish it) or copy it
-        if (!warp_wait_bounded(txbar, ntt & 1u, abort_flag, lim, SITE_TXMSG, kClusterScope)) break;
-        ++ntt;
-        const bool tload = (*tx_msg & 1u) != 0u;
+        // (without an exchange slot, always compute)
+        bool tload = false;
+        if (tx != nullptr) {
+          if (!warp_wait_bounded(txbar, ntt & 1u, abort_flag, lim, SITE_TXMSG, kClusterScope)) break;
+          ++ntt;
+          tload = (*tx_msg & 1u) != 0u;
+        }
         const int t_row = m * (kBM * CG) + int(rank) * kBM + row;
         if (!tload) {
           if (!warp_wait_bounded(tfull, ntc & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
@@ -582,6 +592,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           __nv_bfloat16* const t_dst =
               a.t_out != nullptr && t_row < a.M ? a.t_out + size_t(t_row) * size_t(a.r_pad) : nullptr;
           __nv_bfloat16* const x_dst = tx != nullptr ? tx->t + size_t(t_row) * size_t(a.r_pad) : nullptr;
+#pragma unroll 1
           for (int col = 0; col < a.r_pad; col += 16) {
             uint32_t v[16];
             tmem_ld_x16(tmem + lane_base + t_col + uint32_t(col), v);
@@ -623,6 +634,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           // its flag complete): copy this thread's row into shared memory
           if (!wait_word_bounded(&tx->flags[m], tx_full, abort_flag, lim, SITE_TXFLAG)) break;
           const __nv_bfloat16* const src = tx->t + size_t(t_row) * size_t(a.r_pad);
+          // kept rolled: unrolled, this loop took the kernel from about 100 to
+          // 210 registers and the tiny forward 1-2 us slower
+#pragma unroll 1
           for (int col = 0; col < a.r_pad; col += 16) {
             const uint4 lo = ld_global_cg_v4(src + col);
             const uint4 hi = ld_global_cg_v4(src + col + 8);

@@ -258,9 +258,9 @@ int max_clusters(Kern kern, int cg, uint32_t smem, int sm_count) {
   return n;
 }
 
-template <int BN, bool MN, int RCW, int CG>
+template <int BN, bool MN, int RCW, int CG, bool TX>
 lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
-  auto kern = fused_lora_kernel<BN, MN, RCW, CG>;
+  auto kern = fused_lora_kernel<BN, MN, RCW, CG, TX>;
   if (!ensure_smem_attr(kern, c.smem)) return LORA_ERR_CUDA;
   const int64_t tiles = int64_t(c.args.num_m) * c.args.num_n;
   const int clusters = int(std::min<int64_t>(tiles, max_clusters(kern, CG, c.smem, sm_count)));
@@ -269,20 +269,28 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
                    maps[1], maps[2], maps[3], maps[4], c.args);
 }
 
+// The forward instances with (TX) and without an exchange slot.
+template <int BN, int RCW, int CG>
+lora_status_t launch_fused_fwd(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
+  return c.args.tx != nullptr ? launch_fused_t<BN, false, RCW, CG, true>(maps, c, sm_count, st)
+                              : launch_fused_t<BN, false, RCW, CG, false>(maps, c, sm_count, st);
+}
+
 template <bool MN, int CG>
 lora_status_t launch_fused_cg(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
   if constexpr (MN) {  // the dX form has no rank chunks in shared memory
-    return c.BN == 256 ? launch_fused_t<256, true, 64, CG>(maps, c, sm_count, st)
-                       : launch_fused_t<128, true, 64, CG>(maps, c, sm_count, st);
+    return c.BN == 256 ? launch_fused_t<256, true, 64, CG, false>(maps, c, sm_count, st)
+                       : launch_fused_t<128, true, 64, CG, false>(maps, c, sm_count, st);
+  } else {
+    if (c.BN == 256) {
+      if (c.RCW == 16) return launch_fused_fwd<256, 16, CG>(maps, c, sm_count, st);
+      if (c.RCW == 32) return launch_fused_fwd<256, 32, CG>(maps, c, sm_count, st);
+      return launch_fused_fwd<256, 64, CG>(maps, c, sm_count, st);
+    }
+    if (c.RCW == 16) return launch_fused_fwd<128, 16, CG>(maps, c, sm_count, st);
+    if (c.RCW == 32) return launch_fused_fwd<128, 32, CG>(maps, c, sm_count, st);
+    return launch_fused_fwd<128, 64, CG>(maps, c, sm_count, st);
   }
-  if (c.BN == 256) {
-    if (c.RCW == 16) return launch_fused_t<256, MN, 16, CG>(maps, c, sm_count, st);
-    if (c.RCW == 32) return launch_fused_t<256, MN, 32, CG>(maps, c, sm_count, st);
-    return launch_fused_t<256, MN, 64, CG>(maps, c, sm_count, st);
-  }
-  if (c.RCW == 16) return launch_fused_t<128, MN, 16, CG>(maps, c, sm_count, st);
-  if (c.RCW == 32) return launch_fused_t<128, MN, 32, CG>(maps, c, sm_count, st);
-  return launch_fused_t<128, MN, 64, CG>(maps, c, sm_count, st);
 }
 
 template <bool MN>

@@ -265,8 +265,10 @@ static lora_status_t fwd_run(const void* X, const void* W, const void* A, const 
   c.args.scale = scale;
   c.args.out = reinterpret_cast<__nv_bfloat16*>(Y);
   c.args.t_out = Tws;
-  // with an exchange slot, the schedule that shares T between clusters
-  TxSlot* const tx = c.tx_fits ? tx_slot_for(st) : nullptr;
+  // with an exchange slot, the seeded schedule that shares T between
+  // clusters (other schedules would gain nothing from the exchange: the
+  // runs of an M block start together)
+  TxSlot* const tx = c.tx_fits && c.seeded_l > 0 ? tx_slot_for(st) : nullptr;
   c.args.tx = tx;
   const bool seeded = tx != nullptr && c.seeded_l > 0;
   c.args.run_l = seeded ? c.seeded_l : c.run_l_plain;

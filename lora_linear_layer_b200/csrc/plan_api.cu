@@ -50,7 +50,7 @@ lora_status_t lora_plan(int64_t M, int64_t d_in, int64_t d_out, int32_t r, int32
     out->fwd_stages = c.stages;
     out->fwd_run_l = c.args.run_l;
     out->fwd_seeded = c.args.seeded;
-    out->fwd_tx = c.tx_fits ? 1 : 0;
+    out->fwd_tx = c.tx_fits && c.seeded_l > 0 ? 1 : 0;
     out->fwd_num_m = c.args.num_m;
     out->fwd_num_n = c.args.num_n;
     out->fwd_splits = 1;

@@ -55,6 +55,9 @@ def test_peak_follows_the_length_of_the_timed_region():
     assert bench.pick_peak(peaks, 0.999) == (1654.6, False)
     assert bench.pick_peak(peaks, 1.0) == (1410.9, True)          # seconds at the power cap: sustained
     assert bench.pick_peak({}, 0.01)[0] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    # a short region that nevertheless ran at the power cap takes the sustained figure
+    assert bench.pick_peak(peaks, 0.15, {"reasons": ["sw_power_cap"]}) == (1410.9, True)
+    assert bench.pick_peak(peaks, 0.15, {"reasons": []}) == (1654.6, False)
 
 
 def test_clock_normalised_time():
