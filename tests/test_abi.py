@@ -272,3 +272,66 @@ def test_ctypes_structs_mirror_the_header(built_lib):
         want = [(n, c[t]) for n, t in structs[cname]]
         assert [(n, t) for n, t in cls._fields_] == want, cname
     assert ctypes.sizeof(L._Plan) == 96 and ctypes.sizeof(L._FwdDesc) == 64 and ctypes.sizeof(L._MergeDesc) == 48
+
+
+def _call(so, name, *args):
+    return int(getattr(so, name)(*args))
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,ptr_fix", [
+    (256, 512, 512, 16, None),            # valid: both reach the device step (no GPU here)
+    (-1, 512, 512, 16, None),             # bad size
+    (256, 516, 512, 16, None),
+    (256, 512, 512, 12, None),            # bad rank
+    (256, 512, 512, 16, ("null", 1)),     # NULL W
+    (256, 512, 512, 16, ("odd", 2)),      # A not 16-byte aligned
+    (256, 512, 512, 16, ("alias", 4)),    # Y on top of X
+])
+def test_scaled_forms_apply_the_alpha_forms_rules(built_lib, M, d_in, d_out, r, ptr_fix):
+    """Each *_scaled entry point takes `scale` where its alpha form takes
+    alpha and otherwise validates exactly the same way: the same status for
+    valid and invalid arguments (fake pointers, never dereferenced; on a
+    machine without a GPU a valid call stops at the device check)."""
+    L = built_lib
+    so = L.lib()
+    p = _ptrs(10)
+    if ptr_fix is not None:
+        kind, i = ptr_fix
+        p[i] = 0 if kind == "null" else (p[i] + 8 if kind == "odd" else p[0])
+    X, W, A, B, Y, dY, dX, dA, dB, ws = (ctypes.c_void_p(v) for v in p)
+    f = ctypes.c_float(32.0)
+    need = L.lora_bwd_workspace_size(max(M, 0), d_in, d_out, r) if M >= 0 and r in (8, 16, 128) else 1 << 20
+    pairs = [
+        (("lora_fwd", X, W, A, B, Y, M, d_in, d_out, r, f, None),
+         ("lora_fwd_scaled", X, W, A, B, Y, M, d_in, d_out, r, f, None)),
+        (("lora_fwd_save", X, W, A, B, Y, M, d_in, d_out, r, f, ws, need, None),
+         ("lora_fwd_save_scaled", X, W, A, B, Y, M, d_in, d_out, r, f, ws, need, None)),
+        (("lora_bwd_ex", X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, f, ws, need, 0, None),
+         ("lora_bwd_scaled", X, W, A, B, dY, dX, dA, dB, M, d_in, d_out, r, f, ws, need, 0, None)),
+        (("lora_bwd_grads", X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 0, None),
+         ("lora_bwd_grads_scaled", X, A, B, dY, dA, dB, M, d_in, d_out, r, f, ws, need, 0, None)),
+        (("lora_merge", W, A, B, Y, d_out, d_in, r, f, None),
+         ("lora_merge_scaled", W, A, B, Y, d_out, d_in, r, f, None)),
+    ]
+    for a, b in pairs:
+        ca, cb = _call(so, *a), _call(so, *b)
+        assert ca == cb, (a[0], L.STATUS.get(ca), b[0], L.STATUS.get(cb))
+    # an unknown flag bit is refused by the scaled backward as by lora_bwd_ex
+    assert L.STATUS[_call(so, "lora_bwd_scaled", X, W, A, B, dY, dX, dA, dB, 256, 512, 512, 16, f, ws,
+                          1 << 26, 1 << 7, None)] == "LORA_ERR_FLAGS"
+
+
+def test_scaled_batched_forms_apply_the_alpha_forms_rules(built_lib):
+    L = built_lib
+    so = L.lib()
+    p = _ptrs(12)
+    f = ctypes.c_float(2.0)
+    fwd = (L._FwdDesc * 2)(L._FwdDesc(*p[0:5], 256, 512, 512), L._FwdDesc(*p[5:10], 128, 512, 520))
+    mrg = (L._MergeDesc * 2)(L._MergeDesc(*p[0:4], 512, 512), L._MergeDesc(*p[4:8], 100, 512))  # bad d_out
+    for n in (0, 1, 2, -1):
+        assert _call(so, "lora_fwd_batched", fwd, n, 16, f, None) == _call(so, "lora_fwd_batched_scaled", fwd, n, 16,
+                                                                              f, None)
+        assert _call(so, "lora_merge_batched", mrg, n, 16, f, None) == _call(so, "lora_merge_batched_scaled", mrg,
+                                                                              n, 16, f, None)
+    assert L.STATUS[_call(so, "lora_merge_batched_scaled", mrg, 2, 16, f, None)] == "LORA_ERR_SHAPE"
+    assert L.STATUS[_call(so, "lora_fwd_batched_scaled", fwd, 2, 12, f, None)] == "LORA_ERR_RANK"
