@@ -36,6 +36,13 @@
 // runs.  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM
 // owner, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)...).
 //
+// BN = 224 (forward, CTA pairs, r_pad <= 32): the pair fold.  The odd CTA's
+// Q slot holds the tile's W rows [128, 224) and 32 rows of U, so the
+// tile's one N = 256 MMA per K step yields the base product in accumulator
+// columns [0, 224) and T in [224, 256): no separate N = r products, at the
+// price of 32 of every 256 columns.  Used where few tiles per pair would
+// each compute T.
+//
 // CG = 2 runs each tile on a CTA pair (a cluster of two, cta_group::2):
 // each CTA holds its own 128 rows of P and half of the Q/U/V rows, the even
 // CTA issues every MMA (M = 256) for both, and each CTA keeps its 128 rows
@@ -55,6 +62,10 @@ namespace lora {
 constexpr int kBM = 128;          // rows per CTA (UMMA M per CTA)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr int kFusedThreads = 192;
+// Pair tile with T folded into the base product: 224 output columns and the
+// 32 columns of T in one N = 256 MMA (forward, CTA pairs, r_pad <= 32).
+constexpr int kPairFoldBN = 224;
+constexpr int kPairFoldT = 32;
 constexpr int kEpCols = 32;                    // output columns per epilogue store
 constexpr uint32_t kEpBufBytes = 32u * kEpCols * 2u;  // one warp's 32 rows, 64-byte swizzle
 
@@ -82,11 +93,14 @@ struct FusedLayout {
   uint32_t off_st, off_ep, off_bar, total;
   __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages,
                                   int ep_bufs) {
-    const int bnc = BN / CG;            // Q / V rows held by this CTA
+    // Q / V rows held by this CTA (the 224-wide pair tile: 128 in each CTA,
+    // the odd CTA's last 32 of them rows of U)
+    const int bnc = BN == kPairFoldBN ? 128 : BN / CG;
     p_bytes = kBM * kBK * 2;
     q_bytes = uint32_t(bnc * kBK * 2);
-    // the dX form streams its rank-side operands through the ring
-    u_bytes = mn ? 0u : uint32_t((r_pad / CG) * 128);
+    // the dX form streams its rank-side operands through the ring; the
+    // 224-wide pair tile holds U in its Q slot
+    u_bytes = (mn || BN == kPairFoldBN) ? 0u : uint32_t((r_pad / CG) * 128);
     stage_bytes = p_bytes + q_bytes + u_bytes;
     // V (the up-projection's rank-side operand of one N tile) travels
     // through the ring as one more stage per tile: all its chunks fit in a
@@ -265,14 +279,21 @@ template <int BN, bool MN, int RCW, int CG, bool TX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_lora_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
-                      const __grid_constant__ CUtensorMap tmO, const FusedArgs a) {
-  static_assert(BN == 128 || BN == 256, "BN");
+                      const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmQ2,
+                      const FusedArgs a) {
+  static_assert(BN == 128 || BN == 256 || (BN == kPairFoldBN && CG == 2 && !MN), "BN");
   static_assert(CG == 1 || CG == 2, "CG");
   static_assert(RCW == 16 || RCW == 32 || RCW == 64, "RCW");
   static_assert(!(TX && MN), "the exchange is a forward feature");
   constexpr bool kQmn = MN;             // Q read MN-major
   using G = Group<CG>;
-  constexpr int BNC = BN / CG;          // Q / V rows held by this CTA
+  // 224-wide pair tile (kPairFoldBN): the even CTA holds Q rows [0, 128) of
+  // the tile, the odd one Q rows [128, 224) and U's rows, so one N = 256
+  // MMA puts the base product in accumulator columns [0, 224) and T in
+  // [224, 256) (the single-CTA fold's idea on the pair; tmQ2 is Q with a
+  // 96-row box)
+  constexpr bool kPF = BN == kPairFoldBN;
+  constexpr int BNC = kPF ? 128 : BN / CG;  // Q / V rows held by this CTA
   constexpr uint32_t kRSwz = RCW == 16 ? SWZ_32B : RCW == 32 ? SWZ_64B : SWZ_128B;
   constexpr uint32_t kRSpan = RCW * 2;  // bytes per swizzled rank row
   constexpr bool kClusterScope = CG > 1;
@@ -331,6 +352,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmU);
     tma_prefetch_desc(&tmV);
+    if constexpr (kPF) tma_prefetch_desc(&tmQ2);
   }
   if (warp == 2 && lane == 0) tma_prefetch_desc(&tmO);
   if (warp == 1) G::alloc(smem_addr(tmem_slot), 512);
@@ -351,8 +373,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   // if two BN-wide accumulators and r_pad columns fit in 512, else it
   // borrows the other accumulator.
   constexpr bool kFold = CG == 1 && BN == 128 && !MN;
-  const uint32_t acc_stride = kFold ? uint32_t(BN + a.r_pad) : uint32_t(BN);
-  const bool borrow = !MN && !kFold && (2 * BN + a.r_pad) > 512;
+  const uint32_t acc_stride = kFold ? uint32_t(BN + a.r_pad) : kPF ? uint32_t(BN + kPairFoldT) : uint32_t(BN);
+  const bool borrow = !MN && !kFold && !kPF && (2 * BN + a.r_pad) > 512;
   const int nk = (a.K + kBK - 1) / kBK;
   // dX: K blocks [nk, nk_all) hold the rank-side product dT A
   const int nk_all = MN ? nk + (a.r_pad + kBK - 1) / kBK : nk;
@@ -381,7 +403,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
         const uint32_t bytes = L.p_bytes + L.q_bytes + (ttile ? L.u_bytes : 0u);
         const int row0 = m * (kBM * CG) + int(rank) * kBM;
-        const int qrow0 = n * BN + int(rank) * BNC;
+        const int qrow0 = n * BN + int(rank) * BNC;  // (the pair fold's odd CTA: its first W row)
         for (int kb = 0; kb < nk_all; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, lim, SITE_EMPTY, kClusterScope)) {
             ok = false;
@@ -397,14 +419,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           if (!MN || kb < nk) {
             const int k0 = kb * kBK;
             G::load(st, &tmP, fb, k0, row0);
-            if (!kQmn) {
+            if (kPF) {
+              if (rank == 0) {
+                G::load(st + L.p_bytes, &tmQ, fb, k0, qrow0);
+              } else {
+                G::load(st + L.p_bytes, &tmQ2, fb, k0, qrow0);
+                G::load(st + L.p_bytes + uint32_t((128 - kPairFoldT) * 128), &tmU, fb, k0, 0);
+              }
+            } else if (!kQmn) {
               G::load(st + L.p_bytes, &tmQ, fb, k0, qrow0);
             } else {
 #pragma unroll
               for (int i = 0; i < BNC / 64; ++i)
                 G::load(st + L.p_bytes + uint32_t(i) * 8192u, &tmQ, fb, qrow0 + 64 * i, k0);
             }
-            if (ttile) G::load(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, int(rank) * u_rows);
+            if (!kPF && ttile) G::load(st + L.p_bytes + L.q_bytes, &tmU, fb, k0, int(rank) * u_rows);
           } else {
             // dX tail: dT and A in place of dY and W (columns of dT and rows
             // of A past r_pad come from the tensor maps' zero fill)
@@ -433,10 +462,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer ----
     if (lane == 0 && leader) {
-      const uint32_t id_base = idesc_bf16(kBM * CG, BN, false, kQmn);
+      const uint32_t id_base = idesc_bf16(kBM * CG, kPF ? BN + kPairFoldT : BN, false, kQmn);
       const uint32_t id_tail = idesc_bf16(kBM * CG, BN, false, true);  // dX: V = A is MN-major
       const uint32_t id_t = idesc_bf16(kBM * CG, a.r_pad, false, false);
-      const uint32_t id_up = idesc_bf16(kBM * CG, BN, false, MN);
+      const uint32_t id_up = idesc_bf16(kBM * CG, kPF ? BN + kPairFoldT : BN, false, MN);
       const uint32_t id_fold = idesc_bf16(kBM * CG, BN + a.r_pad, false, false);
       TileSched sch(a, n_clusters, cluster_id);
       int m, n, prev_m = -1, stage = 0;
@@ -472,7 +501,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const uint32_t b = tcount & 1u;
         if (!wait_bounded(accempty0 + 8u * b, next_acc_parity(b), abort_flag, lim, SITE_ACCEMPTY, kClusterScope))
           break;
-        uint32_t t_col = kFold ? b * acc_stride + BN : 2u * BN;
+        uint32_t t_col = (kFold || kPF) ? b * acc_stride + BN : 2u * BN;
         if (tcomp && borrow) {
           const uint32_t ob = b ^ 1u;
           if (!wait_bounded(accempty0 + 8u * ob, next_acc_parity(ob), abort_flag, lim, SITE_ACCEMPTY,
@@ -511,7 +540,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 G::mma(d_acc, smem_desc(st + kk * 32u, 16u, 1024u, SWZ_128B),
                        smem_desc(sq + kk * 2048u, 8192u, 1024u, SWZ_128B), id_tail, 1u);
             }
-            if constexpr (kWithT && !kFold) {
+            if constexpr (kWithT && !kFold && !kPF) {
               const uint32_t su = sq + L.q_bytes;
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk)
@@ -586,7 +615,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           if (!warp_wait_bounded(tfull, ntc & 1u, abort_flag, lim, SITE_TFULL, kClusterScope)) break;
           ++ntc;
           tc_fence_after();
-          const uint32_t t_col = kFold ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
+          const uint32_t t_col = (kFold || kPF) ? b * acc_stride + BN : borrow ? (b ^ 1u) * BN : 2u * BN;
           // every tile that computes T stores it for the backward when asked
           // (the same values whichever tile of the M block does)
           __nv_bfloat16* const t_dst =

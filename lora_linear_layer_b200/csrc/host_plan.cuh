@@ -39,6 +39,7 @@ struct FusedCfg {
   int seeded_l;              // seeded schedule's run length when the launch gets a slot (0: runs) ...
   double seeded_cost;
   int run_l_plain;           // ... and the run length without one (runs cover every N tile)
+  double model_cost;         // modelled makespan in 256 x 256 pair-tile times (CTA-pair tiles only; else 0)
   FusedArgs args;
 };
 
@@ -58,7 +59,8 @@ void tile_override(int& BN, int& CG) {
   const char* e = std::getenv("LORA_B200_FUSED_TILE");
   if (e == nullptr) return;
   int b = 0, g = 0;
-  if (std::sscanf(e, "%d,%d", &b, &g) == 2 && (b == 128 || b == 256) && (g == 1 || g == 2)) {
+  if (std::sscanf(e, "%d,%d", &b, &g) == 2 &&
+      (((b == 128 || b == 256) && (g == 1 || g == 2)) || (b == kPairFoldBN && g == 2))) {
     BN = b;
     CG = g;
   }
@@ -79,12 +81,12 @@ int run_override() {
   return v >= 0 && v <= 4096 ? v : -1;
 }
 
-bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, FusedCfg& c) {
+// The plan for one tile choice: (fBN, fCG) forced, or 0, 0 to choose.
+bool pick_fused_tile(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, int fBN, int fCG,
+                     FusedCfg& c) {
   c.r_pad = r_pad_of(r);
   c.RCW = rcw_of(c.r_pad);
   c.n_rchunks = (c.r_pad + c.RCW - 1) / c.RCW;
-  int fBN, fCG;
-  tile_override(fBN, fCG);
   // Candidates in order of preference: 256-wide tiles first (least operand
   // traffic per flop); CTA pairs first for long contractions, single CTAs
   // first for K <= 1024 (measured faster there: 8192x512x512 16.4 vs
@@ -96,16 +98,18 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   // case: 512x4096x4096 43.0 vs 41.0 us).  LORA_B200_FUSED_TILE can still
   // force a 128-wide pair.
   const bool short_k = K <= 1024;
-  const int cands[4][2] = {{256, short_k ? 1 : 2}, {256, short_k ? 2 : 1}, {128, 1}, {128, 2}};
+  const int cands[5][2] = {
+      {256, short_k ? 1 : 2}, {256, short_k ? 2 : 1}, {128, 1}, {128, 2}, {kPairFoldBN, 2}};
   c.BN = 0;
   for (int pass = 0; pass < 2 && c.BN == 0; ++pass) {  // pass 1 ignores an infeasible override
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 5; ++i) {
       const int BN = cands[i][0], CG = cands[i][1];
       const bool forced = pass == 0 && fBN != 0;
       if (forced && (BN != fBN || CG != fCG)) continue;
-      if (!forced && i == 3) break;  // the 128-wide pair only when forced
+      if (!forced && i >= 3) break;  // the 128-wide pair and the pair fold only when forced (or chosen below)
+      if (BN == kPairFoldBN && (mn || c.r_pad > kPairFoldT)) continue;  // forward only, T in 32 columns
       const int S = fused_stages(BN, CG, mn, c.RCW, c.r_pad, c.n_rchunks, 1);
-      if (S < (BN == 256 ? 3 : 2)) continue;
+      if (S < (BN >= 224 ? 3 : 2)) continue;
       const int64_t tiles = ((M + 128 * CG - 1) / (128 * CG)) * ((N + BN - 1) / BN);
       const bool fills = double(tiles) >= 0.8 * double(sm_count / CG);
       if (forced || fills || i == 2) {
@@ -214,9 +218,56 @@ bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, F
   const int ro = run_override();
   if (ro >= 0) c.seeded_l = 0;
   c.run_l_plain = ro >= 0 ? ro : best_l;
+  if (c.BN == kPairFoldBN) {
+    // T comes with the base product: no exchange, and single-tile runs
+    // dealt round-robin (as the dX form) keep the tiles in flight on a few
+    // M blocks
+    c.tx_fits = false;
+    c.seeded_l = 0;
+    c.run_l_plain = ro >= 0 ? ro : 1;
+  }
   a.run_l = c.seeded_l > 0 ? c.seeded_l : c.run_l_plain;
   a.seeded = c.seeded_l > 0 ? 1 : 0;
   a.wait_limit_ns = kWaitLimitNs;
+  // modelled makespan in 256 x 256 pair-tile times, for the choice below
+  c.model_cost = 0.0;
+  if (c.CG == 2 && c.BN == kPairFoldBN) {
+    // a fold tile computes 256 columns for 224 of output: 1.15 tile times
+    // fits the same-box measurements (512 x 8192^2: fold 0.84 of the
+    // 256-wide pair's time, 1024 x 8192^2 0.93, 2048 x 8192^2 1.04,
+    // 512 x 4096 x 14336 1.03-1.14)
+    c.model_cost = 1.15 * double((int64_t(num_m) * num_n + clusters - 1) / clusters);
+  } else if (c.CG == 2 && c.BN == 256 && !mn) {
+    if (c.seeded_l > 0) {
+      c.model_cost = c.seeded_cost;
+    } else if (c.run_l_plain > 0) {
+      const int64_t runs = int64_t(num_m) * ((num_n + c.run_l_plain - 1) / c.run_l_plain);
+      c.model_cost = double((runs + clusters - 1) / clusters) * (c.run_l_plain + 0.5);
+    } else {
+      c.model_cost = double((int64_t(num_m) * num_n + clusters - 1) / clusters) + 0.5;
+    }
+  }
+  return true;
+}
+
+// The forward's tile: as pick_fused_tile chooses, or, where that is the
+// 256-wide pair, the 224-wide pair fold when its grid fills the pairs and its
+// modelled makespan is at least 10% shorter.  The fold pays no separate T
+// products (a T tile of the 256-wide pair costs about 1.5 tile times: the
+// N = r products take as long as N = 128 ones), but every fold tile spends
+// 32 of its 256 columns on T, and its 224-wide grid quantises differently:
+// it wins where few tiles per pair each compute T (512 x 8192 x 8192: 64
+// pair tiles with T against 74 fold tiles), and loses where the exchange or
+// longer runs leave one T per pair (8192 x 4096 x 4096: 7.5 against 10.4).
+bool pick_fused(int64_t M, int64_t N, int64_t K, int r, bool mn, int sm_count, FusedCfg& c) {
+  int fBN, fCG;
+  tile_override(fBN, fCG);
+  if (!pick_fused_tile(M, N, K, r, mn, sm_count, fBN, fCG, c)) return false;
+  if (fBN != 0 || mn || c.BN != 256 || c.CG != 2 || r_pad_of(r) > kPairFoldT) return true;
+  FusedCfg pf;
+  if (!pick_fused_tile(M, N, K, r, mn, sm_count, kPairFoldBN, 2, pf) || pf.BN != kPairFoldBN) return true;
+  const int64_t pf_tiles = int64_t(pf.args.num_m) * pf.args.num_n;
+  if (double(pf_tiles) >= 0.8 * double(sm_count / 2) && pf.model_cost <= 0.9 * c.model_cost) c = pf;
   return true;
 }
 
@@ -258,6 +309,7 @@ int max_clusters(Kern kern, int cg, uint32_t smem, int sm_count) {
   return n;
 }
 
+// maps: P, Q, U, V, OUT and the pair fold's second Q map (any valid map otherwise)
 template <int BN, bool MN, int RCW, int CG, bool TX>
 lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_count, cudaStream_t st) {
   auto kern = fused_lora_kernel<BN, MN, RCW, CG, TX>;
@@ -266,7 +318,7 @@ lora_status_t launch_fused_t(const CUtensorMap* maps, const FusedCfg& c, int sm_
   const int clusters = int(std::min<int64_t>(tiles, max_clusters(kern, CG, c.smem, sm_count)));
   const dim3 cl(unsigned(CG), 1, 1);
   return launch_ex("fused", kern, dim3(unsigned(clusters * CG)), dim3(kFusedThreads), c.smem, st, &cl, maps[0],
-                   maps[1], maps[2], maps[3], maps[4], c.args);
+                   maps[1], maps[2], maps[3], maps[4], maps[5], c.args);
 }
 
 // The forward instances with (TX) and without an exchange slot.
@@ -282,6 +334,11 @@ lora_status_t launch_fused_cg(const CUtensorMap* maps, const FusedCfg& c, int sm
     return c.BN == 256 ? launch_fused_t<256, true, 64, CG, false>(maps, c, sm_count, st)
                        : launch_fused_t<128, true, 64, CG, false>(maps, c, sm_count, st);
   } else {
+    if constexpr (CG == 2) {
+      if (c.BN == kPairFoldBN)  // r_pad <= 32, no exchange
+        return c.RCW == 16 ? launch_fused_t<kPairFoldBN, false, 16, 2, false>(maps, c, sm_count, st)
+                           : launch_fused_t<kPairFoldBN, false, 32, 2, false>(maps, c, sm_count, st);
+    }
     if (c.BN == 256) {
       if (c.RCW == 16) return launch_fused_fwd<256, 16, CG>(maps, c, sm_count, st);
       if (c.RCW == 32) return launch_fused_fwd<256, 32, CG>(maps, c, sm_count, st);

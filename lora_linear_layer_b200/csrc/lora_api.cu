@@ -273,13 +273,18 @@ static lora_status_t fwd_run(const void* X, const void* W, const void* A, const 
   const bool seeded = tx != nullptr && c.seeded_l > 0;
   c.args.run_l = seeded ? c.seeded_l : c.run_l_plain;
   c.args.seeded = seeded ? 1 : 0;
-  CUtensorMap maps[5];
-  const uint32_t bnc = uint32_t(c.BN / c.CG);
+  CUtensorMap maps[6];
+  // Q and V rows per CTA, and U's rows per CTA; the pair fold's odd CTA
+  // loads 96 rows of W (maps[5]) and 32 of A
+  const bool pf = c.BN == kPairFoldBN;
+  const uint32_t bnc = pf ? 128u : uint32_t(c.BN / c.CG);
+  const uint32_t u_box = pf ? uint32_t(kPairFoldT) : uint32_t(c.r_pad / c.CG);
   if (!make_map(&maps[0], X, d_in, M, d_in, 64, 128, 128) ||
       !make_map(&maps[1], W, d_in, d_out, d_in, 64, bnc, 128) ||
-      !make_map(&maps[2], A, d_in, r, d_in, 64, uint32_t(c.r_pad / c.CG), 128) ||
+      !make_map(&maps[2], A, d_in, r, d_in, 64, u_box, 128) ||
       !make_map(&maps[3], B, r, d_out, r, c.RCW, bnc, c.RCW * 2) ||
-      !make_map(&maps[4], Y, d_out, M, d_out, kEpCols, 32, kEpCols * 2))
+      !make_map(&maps[4], Y, d_out, M, d_out, kEpCols, 32, kEpCols * 2) ||
+      !make_map(&maps[5], W, d_in, d_out, d_in, 64, pf ? uint32_t(128 - kPairFoldT) : bnc, 128))
     return LORA_ERR_CUDA;
   return launch_fused<false>(maps, c, sm_count, st);
 }
@@ -481,13 +486,14 @@ static lora_status_t launch_bwd_dx(const void* W, const void* A, const void* dY,
     if (!pick_fused(M, d_in, d_out, r, true, sm_count, c)) return LORA_ERR_RANK;
     c.args.scale = 1.0f;
     c.args.out = reinterpret_cast<__nv_bfloat16*>(dX);
-    CUtensorMap maps[5];
+    CUtensorMap maps[6];
     if (!make_map(&maps[0], dY, d_out, M, d_out, 64, 128, 128) ||
         !make_map(&maps[1], W, d_in, d_out, d_in, 64, 64, 128) ||
         !make_map(&maps[2], dTws, r_pad, M, r_pad, 64, 128, 128) ||
         !make_map(&maps[3], A, d_in, r, d_in, 64, 64, 128) ||
         !make_map(&maps[4], dX, d_in, M, d_in, kEpCols, 32, kEpCols * 2))
       return LORA_ERR_CUDA;
+    maps[5] = maps[1];  // (unused by the dX form)
     if ((s = launch_fused<true>(maps, c, sm_count, st)) != LORA_OK) return s;
   }
   return LORA_OK;

@@ -100,7 +100,13 @@ def _check_plan(p, M, d_in, d_out, r, forced_tile=None, forced_run=None):
     for k in ("fwd_smem", "bwd1_smem", "bwd2_smem", "dx_smem"):
         assert 0 < p[k] <= SMEM_MAX, (k, where)
     if p["fwd_kind"] == 0:
-        assert p["fwd_bn"] in (128, 256) and p["fwd_cg"] in (1, 2) and p["fwd_stages"] >= 2, where
+        assert p["fwd_bn"] in (128, 224, 256) and p["fwd_cg"] in (1, 2) and p["fwd_stages"] >= 2, where
+        if p["fwd_bn"] == 224:
+            # the pair fold: CTA pairs, T in the base product's last 32 columns, no exchange
+            assert p["fwd_cg"] == 2 and r <= 32 and p["fwd_tx"] == 0 and p["fwd_seeded"] == 0, where
+            assert p["fwd_stages"] >= 3, where
+            if forced_run is None:
+                assert p["fwd_run_l"] == 1, where
         assert p["fwd_splits"] == 1, where
         assert p["fwd_num_m"] == math.ceil(M / (128 * p["fwd_cg"])), where
         assert p["fwd_num_n"] == math.ceil(d_out / p["fwd_bn"]), where
@@ -143,13 +149,14 @@ def test_every_plan_fits_and_covers(built_lib, monkeypatch, r):
         _check_plan(built_lib.lora_plan(M, d_in, d_out, r), M, d_in, d_out, r)
 
 
-@pytest.mark.parametrize("tile", [(256, 2), (256, 1), (128, 2), (128, 1)])
+@pytest.mark.parametrize("tile", [(256, 2), (256, 1), (128, 2), (128, 1), (224, 2)])
 def test_forced_tiles_fit(built_lib, monkeypatch, tile):
     """Every tile configuration the tests force is launchable for every rank
     (enough shared memory for a pipeline) and is the one used, except 256-wide
-    single-CTA tiles at r = 128: they leave room for two stages, the planner
-    wants three for 256-wide tiles, and the override falls back to the
-    automatic choice for the shape."""
+    single-CTA tiles at r = 128 (they leave room for two stages, the planner
+    wants three for 256-wide tiles) and the 224-wide pair fold above r = 32
+    (T has 32 columns of the accumulator): there the override falls back to
+    the automatic choice for the shape."""
     for v in ("LORA_B200_FUSED_RUN", "LORA_B200_SPLITK", "LORA_B200_TX", "LORA_B200_SEEDED_L"):
         monkeypatch.delenv(v, raising=False)
     for r, M, d in itertools.product(RS, (1, 1000, 8192), (64, 1032, 4096)):
@@ -157,9 +164,9 @@ def test_forced_tiles_fit(built_lib, monkeypatch, tile):
         auto = built_lib.lora_plan(M, d, d, r)
         monkeypatch.setenv("LORA_B200_FUSED_TILE", f"{tile[0]},{tile[1]}")
         p = built_lib.lora_plan(M, d, d, r)
-        if tile == (256, 1) and r == 128:
+        if (tile == (256, 1) and r == 128) or (tile == (224, 2) and r > 32):
             _check_plan(p, M, d, d, r)
-            assert (p["fwd_bn"], p["fwd_cg"]) == (auto["fwd_bn"], auto["fwd_cg"]) != (256, 1)
+            assert (p["fwd_bn"], p["fwd_cg"]) == (auto["fwd_bn"], auto["fwd_cg"]) != tile
         else:
             _check_plan(p, M, d, d, r, forced_tile=tile)
 
@@ -196,6 +203,15 @@ def test_named_workloads(built_lib, monkeypatch):
     assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_seeded"]) == (0, 256, 2, 2, 1)
     p = built_lib.lora_plan(128, 4096, 4096, 16)        # weight-streaming: split contraction
     assert (p["fwd_kind"], p["fwd_splits"]) == (1, 4)
+    # few pair tiles that would each compute T: the 224-wide pair fold (74 tiles
+    # for 74 pairs at 512 x 8192^2), at r <= 32 only
+    for r in (8, 16, 32):
+        p = built_lib.lora_plan(512, 8192, 8192, r)
+        assert (p["fwd_kind"], p["fwd_bn"], p["fwd_cg"], p["fwd_run_l"], p["fwd_num_n"]) == (0, 224, 2, 1, 37), r
+    assert built_lib.lora_plan(512, 8192, 8192, 64)["fwd_bn"] == 256
+    # runs of 2 or 4 with one T each: the 256-wide pair measured as fast or faster
+    for M, d_in, d_out in ((1024, 8192, 8192), (2048, 8192, 8192), (512, 4096, 14336), (2048, 4096, 4096)):
+        assert built_lib.lora_plan(M, d_in, d_out, 16)["fwd_bn"] == 256, (M, d_in, d_out)
     assert all(v == 0 for v in built_lib.lora_plan(0, 512, 264, 16).values())
 
 
