@@ -481,20 +481,24 @@ def run_ours(args):
 # After a burst of heavy work the part holds a lower SM clock for 0.1-0.2 s
 # (measured: the 512 x 8192^2 forward took 63.5 us cool, 89 us right after
 # 65 calls of 16384 x 8192^2 with the clock at about 1.3 GHz, 72.6 us 50 ms
-# later and 62.5-63.5 us after 0.2 s).  Measurements that follow other work
-# in the same process idle COOL_S first, so that each is taken on a part in
-# the state the burst peak was measured in, whatever ran before it.
+# later and 62.5-63.5 us after 0.2 s).  A measurement that follows heavy
+# work in the same process idles COOL_S first, then warms up, so that it is
+# taken on a part in the state the burst peak was measured in, whatever ran
+# before it.  (Idling before every measurement instead slowed the short ones:
+# the tiny forward's calls, timed right after an idle, took 20 us against
+# 12.3 us.)
 COOL_S = 0.25
-HEAVY_BUSY_S = 0.002       # a sweep point that kept the GPU busy longer than this heats the next one
+HEAVY_BUSY_S = 0.002       # work that kept the GPU busy longer than this heats what follows
 
 
 def _time_events(fn, flush, n, warm=3, cool_s=0.0):
     import torch
+    if cool_s > 0:
+        torch.cuda.synchronize()
+        time.sleep(cool_s)
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
-    if cool_s > 0:
-        time.sleep(cool_s)
     ts = []
     for _ in range(n):
         flush.zero_()
@@ -534,21 +538,32 @@ def _dev_inputs(sh, seed, with_dy=False):
     return X, W, A, B, dY
 
 
+class _Cooled:
+    """Times measurements one after another, each after a COOL_S idle when
+    the one before it kept the GPU busy longer than HEAVY_BUSY_S."""
+
+    def __init__(self):
+        self.busy_s = 0.0
+
+    def time(self, fn, flush, n, warm=3):
+        res = _time_events(fn, flush, n, warm=warm, cool_s=COOL_S if self.busy_s > HEAVY_BUSY_S else 0.0)
+        self.busy_s = res[0] * 1e-6 * (n + warm)
+        return res
+
+
 def measure_sweep(L, flush, P, BW, n=5, warm=2, name_filter=""):
     """lora_fwd on every point of the square sweep: us/call (median, p10,
     p90), TFLOP/s, GB/s of the minimum bytes and the fraction of the binding
     roof (tensor at the burst bf16 peak, or HBM at the copy bandwidth)."""
     import torch
     out = []
-    busy_s = 0.0               # GPU time of the previous point's calls
+    cooled = _Cooled()
     for idx, sh in enumerate(WL.sweep_points()):
         if name_filter and name_filter not in sh.name:
             continue
         X, W, A, B, _ = _dev_inputs(sh, seed=idx)
         Y = torch.empty((sh.M, sh.d_out), dtype=torch.bfloat16, device="cuda")
-        med, p10, p90 = _time_events(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n, warm=warm,
-                                     cool_s=COOL_S if busy_s > HEAVY_BUSY_S else 0.0)
-        busy_s = med * 1e-6 * (n + warm)
+        med, p10, p90 = cooled.time(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n, warm=warm)
         F = flops_fwd(sh.M, sh.d_in, sh.d_out, sh.r)
         by = 2.0 * (sh.M * sh.d_in + sh.d_out * sh.d_in + sh.r * (sh.d_in + sh.d_out) + sh.M * sh.d_out)
         t_roof = max(F / P, by / BW)
@@ -730,15 +745,15 @@ def measure_vs_unfused(L, sh, flush, n):
         y = Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s
         return torch.autograd.grad(y, (Xg, Ag, Bg), dY)
 
-    # every arm starts on a part that has idled COOL_S (the arms run one
-    # after another, the unfused ones heavier)
-    c = COOL_S
-    tf = _time_events(torch_fwd, flush, n, cool_s=c)[0]
-    of = _time_events(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n, cool_s=c)[0]
-    tfb = _time_events(torch_fwd_bwd, flush, n, cool_s=c)[0]
-    tfg = _time_events(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n, cool_s=c)[0]
+    # the arms run one after another, the unfused ones heavier: each follows
+    # an idle when the arm before it was heavy
+    ct = _Cooled().time
+    tf = ct(torch_fwd, flush, n)[0]
+    of = ct(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n)[0]
+    tfb = ct(torch_fwd_bwd, flush, n)[0]
+    tfg = ct(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n)[0]
     tb = max(tfb - tfg, 1e-3)          # the unfused backward alone
-    ob = _time_events(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n, cool_s=c)[0]
+    ob = ct(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n)[0]
     out = {"workload": sh.name, "torch_fwd_us": tf, "ours_fwd_us": of, "fwd_speedup": tf / of,
            "torch_bwd_us": tb, "ours_bwd_us": ob, "bwd_speedup": tb / ob}
     del X, W, A, B, dY, Y, dX, dA, dB, ws, Xg, Ag, Bg
@@ -785,7 +800,7 @@ def run_configs(args, peaks, peak_src):
                                                               if x["bound"] == "tensor"]),
                 "median_roof_frac_hbm": statistics.median([x["roof_frac"] for x in rows if x["bound"] == "hbm"]),
                 "m128": m128, "timing": "median of 5 calls, L2 flushed before each; a point that follows one "
-                                            "that kept the GPU busy over 2 ms is timed after a 0.25 s idle"}
+                                            "that kept the GPU busy over 2 ms idles 0.25 s before its warm-up"}
 
     clocked("sweep", sweep)
     clocked("merge_refresh", lambda: measure_merge(L, flush, 5, BW))
@@ -820,6 +835,7 @@ def run_compare(args):
     import torch
     import lora_linear_layer_b200 as L
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    cooled = _Cooled()
     for sh in compare_shapes():
         if args.sweep_filter and args.sweep_filter not in sh.name:
             continue
@@ -842,17 +858,16 @@ def run_compare(args):
             return torch.autograd.grad(y, (Xg, Ag, Bg), dY)
 
         n = max(5, min(args.steps, 50))
-        c = COOL_S             # every arm starts on a part that has idled (the unfused arms are heavier)
-        tf = _time_events(torch_fwd, flush, n, cool_s=c)[0]
-        of = _time_events(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n, cool_s=c)[0]
+        ct = cooled.time       # an idle before an arm that follows a heavy one (the unfused arms are heavier)
+        tf = ct(torch_fwd, flush, n)[0]
+        of = ct(lambda: L.lora_fwd(X, W, A, B, Y, sh.alpha), flush, n)[0]
         # the unfused backward includes its forward (autograd needs the graph); time the
         # forward alone and subtract it
-        tfb = _time_events(torch_bwd, flush, n, cool_s=c)[0]
-        ob = _time_events(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n, cool_s=c)[0]
+        tfb = ct(torch_bwd, flush, n)[0]
+        ob = ct(lambda: L.lora_bwd(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws), flush, n)[0]
         L.lora_fwd_save(X, W, A, B, Y, sh.alpha, ws)       # T into the workspace, kept by the backward
-        obs = _time_events(lambda: L.lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws, L.LORA_BWD_T_SAVED),
-                           flush, n, cool_s=c)[0]
-        tb = max(tfb - _time_events(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n, cool_s=c)[0], 1e-3)
+        obs = ct(lambda: L.lora_bwd_ex(X, W, A, B, dY, dX, dA, dB, sh.alpha, ws, L.LORA_BWD_T_SAVED), flush, n)[0]
+        tb = max(tfb - ct(lambda: Xg @ W.t() + (Xg @ Ag.t()) @ Bg.t() * s, flush, n)[0], 1e-3)
         print(json.dumps({"point": sh.name, "M": sh.M, "d_in": sh.d_in, "d_out": sh.d_out, "r": sh.r,
                           "torch_fwd_us": tf, "ours_fwd_us": of, "fwd_speedup": tf / of,
                           "torch_bwd_us": tb, "ours_bwd_us": ob, "bwd_speedup": tb / ob,
