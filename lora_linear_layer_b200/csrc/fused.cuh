@@ -94,7 +94,7 @@ struct FusedLayout {
   __host__ __device__ FusedLayout(int BN, int CG, bool mn, int rcw, int r_pad, int n_rchunks, int stages,
                                   int ep_bufs) {
     // Q / V rows held by this CTA (the 224-wide pair tile: 128 in each CTA,
-    // the odd CTA's last 32 of them rows of U)
+    // of which the odd CTA's last 32 are rows of U)
     const int bnc = BN == kPairFoldBN ? 128 : BN / CG;
     p_bytes = kBM * kBK * 2;
     q_bytes = uint32_t(bnc * kBK * 2);
@@ -369,9 +369,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   // T placement.  128-wide single-CTA forward tiles fold T into the base
   // product: U's rows follow Q's rows in the stage, so one MMA with
   // N = BN + r_pad covers both, and each accumulator buffer is BN + r_pad
-  // columns wide with T in its last r_pad.  Otherwise T gets its own columns
-  // if two BN-wide accumulators and r_pad columns fit in 512, else it
-  // borrows the other accumulator.
+  // columns wide with T in its last r_pad.  The 224-wide pair tile does the
+  // same on the pair: its accumulators are 256 columns wide, T in the last
+  // 32 (every MMA of its K loop has N = 256).  Otherwise T gets its own
+  // columns if two BN-wide accumulators and r_pad columns fit in 512, else
+  // it borrows the other accumulator.
   constexpr bool kFold = CG == 1 && BN == 128 && !MN;
   const uint32_t acc_stride = kFold ? uint32_t(BN + a.r_pad) : kPF ? uint32_t(BN + kPairFoldT) : uint32_t(BN);
   const bool borrow = !MN && !kFold && !kPF && (2 * BN + a.r_pad) > 512;
