@@ -368,7 +368,7 @@ lora_status_t lora_check_args(int32_t op, const void* const* ptrs, int32_t n_ptr
 typedef struct {
   int32_t fwd_kind;        /* 0 = tiled kernel (one output tile per CTA or CTA pair),
                               1 = split contraction (the CTAs of a cluster share a tile) */
-  int32_t fwd_bn;          /* output tile width */
+  int32_t fwd_bn;          /* output tile width: 128 or 256; 224 = CTA pair with T folded into an N = 256 MMA */
   int32_t fwd_cg;          /* CTAs per tile (2 = CTA pair) */
   int32_t fwd_stages;      /* pipeline stages */
   int32_t fwd_run_l;       /* tiled: 0 = contiguous ranges, L = runs of L N tiles */
