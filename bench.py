@@ -49,8 +49,9 @@ SUSTAINED_AFTER_S = 1.0
 # the sources the forward kernel's DRAM traffic depends on (kernel and launch
 # configuration / schedule)
 KERNEL_SOURCES = ("lora_linear_layer_b200/csrc/fused.cuh", "lora_linear_layer_b200/csrc/ptx.cuh",
-                  "lora_linear_layer_b200/csrc/common.cuh", "lora_linear_layer_b200/csrc/host_common.cuh",
-                  "lora_linear_layer_b200/csrc/host_plan.cuh", "lora_linear_layer_b200/csrc/lora_api.cu")
+                  "lora_linear_layer_b200/csrc/common.cuh", "lora_linear_layer_b200/csrc/texchange.cuh",
+                  "lora_linear_layer_b200/csrc/host_common.cuh", "lora_linear_layer_b200/csrc/host_plan.cuh",
+                  "lora_linear_layer_b200/csrc/lora_api.cu")
 LAUNCHES_PER_STEP = 5   # fwd 1; bwd: T + dT, dB + dA, dX; merge 1
 
 

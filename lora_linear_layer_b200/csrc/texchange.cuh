@@ -32,7 +32,7 @@ constexpr int kTxSlots = 8;
 constexpr uint32_t kTxMaxBlocks = 4096;        // M blocks per launch
 constexpr size_t kTxElems = size_t(2) << 20;   // bf16 values of s T per slot (4 MiB)
 
-struct TxSlot {
+struct alignas(16) TxSlot {     // 16-byte vector loads and stores of t
   uint32_t done;                 // clusters of the current launch that have finished
   uint32_t pad[3];
   uint32_t flags[kTxMaxBlocks];  // per M block: one bit per epilogue warp that has published its rows
