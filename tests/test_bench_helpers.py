@@ -1,6 +1,7 @@
 """bench.py's host-side helpers (CPU): the algorithmic work it divides by,
 the source hash that keys the recorded DRAM traffic (comment edits keep it,
-code edits change it), and the traffic record's format."""
+code edits change it), the traffic record's format, and when a measurement
+idles first."""
 import os
 import re
 
@@ -64,3 +65,21 @@ def test_clock_normalised_time():
     c = bench._clock_normalised(200.0, {"sm_mhz": 1500.0, "sm_max_mhz": 2000.0})
     assert c["kcycles"] == 300.0 and c["us_at_max_clock"] == 150.0
     assert bench._clock_normalised(200.0, None) is None
+
+
+def test_measurements_idle_only_after_heavy_work(monkeypatch):
+    """_Cooled idles COOL_S before a measurement (before its warm-up) only when
+    the measurement before it kept the GPU busy longer than HEAVY_BUSY_S."""
+    calls = []
+
+    def fake_time_events(fn, flush, n, warm=3, cool_s=0.0):
+        calls.append(cool_s)
+        return fn(), 0.0, 0.0          # the "median" in microseconds
+
+    monkeypatch.setattr(bench, "_time_events", fake_time_events)
+    c = bench._Cooled()
+    light_us = bench.HEAVY_BUSY_S * 1e6 / 20 * 0.5        # 13 calls of it stay under the limit
+    heavy_us = bench.HEAVY_BUSY_S * 1e6 / 13 * 2.0        # 13 calls of it exceed the limit
+    for us in (light_us, light_us, heavy_us, light_us, heavy_us, heavy_us, light_us):
+        c.time(lambda us=us: us, None, 10, warm=3)
+    assert calls == [0.0, 0.0, 0.0, bench.COOL_S, 0.0, bench.COOL_S, bench.COOL_S]
